@@ -1,0 +1,143 @@
+/*
+ * bsg.h -- block-scaled grouped GEMM for NVIDIA B200 (sm_100a): the C ABI of libbsg.so.
+ *
+ * Two operations, both "C = A x B[g]^T with per-row expert routing", computed by hand-written
+ * tcgen05 / TMA / TMEM kernels.  Everything is asynchronous on the caller's CUDA stream; nothing is
+ * allocated, synchronised or retained by a call.  All pointers are CUDA device pointers owned by the
+ * caller unless stated otherwise.  All tensors are dense, row-major, with no padding between rows.
+ *
+ * Error convention (after the argument checks of the FP8 page's host binding, "[flashinfer]
+ * FlashInfer FP8 GEMM 최적화: 윈도우 세그먼트 KG1 프로그램으로 GPU 성능 극대화", section 1): every entry
+ * point validates its arguments on the host before launching anything.  On a violation it returns a
+ * negative bsg_status, launches nothing, and records a one-line description retrievable with
+ * bsg_last_error() (per calling thread).  There is no fallback program and no CPU path.
+ */
+#ifndef BSG_H_
+#define BSG_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* bsg_stream_t; /* a cudaStream_t; NULL is the legacy default stream */
+
+typedef enum {
+  BSG_OK = 0,
+  BSG_ERR_INVALID_ARG = -1,       /* null pointer, non-positive size, bad routing pointer */
+  BSG_ERR_ALIGNMENT = -2,         /* a base pointer or row pitch breaks the 16-byte rule */
+  BSG_ERR_UNSUPPORTED_SHAPE = -3, /* outside the launch contract (M, N, K, G limits) */
+  BSG_ERR_CUDA = -4,              /* a CUDA runtime / driver call failed (message has the code) */
+  BSG_ERR_DEVICE_TIMEOUT = -5     /* a kernel gave up a bounded wait (see bsg_get_device_status) */
+} bsg_status;
+
+/*
+ * FP8 grouped GEMM -- the operation of the FP8 page named above (introduction and section 1):
+ * E4M3 inputs, FP32 scales per 128-element K block, BF16 output, rows grouped by m_indices, with
+ * expert runs free to start inside a 128-row window (section 2).
+ *
+ *   for every row m with g = m_indices[m] in [0, G):
+ *     C[m, n] = bf16( sum_kb a_scale[m, kb] * b_scale[g, n / 128, kb]
+ *                            * sum_{k in block kb} A[m, k] * B[g, n, k] )        (kb = k / 128)
+ *
+ * A        uint8  [M, K]               E4M3 (FN) codes, row-major.
+ * B        uint8  [G, N, K]            E4M3 codes, one K-major [N, K] matrix per expert.
+ * a_scale  float  [M, K/128]           per row and K block.
+ * b_scale  float  [G, ceil(N/128), K/128]  per expert, 128-row block of B[g] and K block.
+ * m_indices int32 [M]                  expert of each row; a value < 0 or >= G means "skip the row:
+ *                                      its C row is left untouched".  May be NULL only when G == 1
+ *                                      (every row goes to expert 0).  Read on the device on every
+ *                                      call, so a captured CUDA graph may be replayed after the
+ *                                      indices (or any operand) change in place.
+ * C        bf16   [M, N]               output; only routed rows are written.
+ * Contract: 1 <= M <= 2^24, 64 <= N <= 2^19, N % 8 == 0, K % 128 == 0, 128 <= K <= 2^20,
+ *           1 <= G <= 4096 (limits from the window program's launch contract, section 2 of the
+ *           page, plus the 16-byte row rules of TMA); A, B, C 16-byte aligned; a_scale, b_scale,
+ *           m_indices 4-byte aligned.
+ * Rows are routed in runs: maximal stretches of consecutive rows with the same expert.  Any order
+ * is correct; sorted (contiguous) runs are the fast case.
+ */
+bsg_status bsg_fp8_grouped_gemm(const void* A, const void* B, const float* a_scale, const float* b_scale,
+                                const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K,
+                                int64_t G, bsg_stream_t stream);
+
+/*
+ * NVFP4 (grouped) GEMM -- the native FP4 x FP4 grouped GEMM of the page "[onnxruntime] ONNX Runtime:
+ * Blackwell (SM120+)에서 NVFP4 QMoE를 위한 네이티브 FP4xFP4 Prefill 최적화", section 1: E2M1 codes
+ * with one E4M3 scale per 16 K elements and an FP32 per-tensor factor.
+ *
+ *   for every row m with g = m_indices[m] in [0, G):
+ *     C[m, n] = bf16( alpha[g] * sum_j sfa[m, j] * sfb[g, n, j]
+ *                                    * sum_{k in block j} A[m, k] * B[g, n, k] )    (j = k / 16)
+ *
+ * A     uint8 [M, K/2]     E2M1 codes, two per byte, the lower-K element in the low nibble.
+ * B     uint8 [G, N, K/2]  same packing, one K-major matrix per expert.
+ * sfa   uint8 [M, K/16]    E4M3 scale codes (non-negative), row-major.
+ * sfb   uint8 [G, N, K/16] E4M3 scale codes (non-negative), row-major.
+ * alpha float [G]          device array: per-expert product of the two per-tensor scales.
+ * m_indices, C             as for bsg_fp8_grouped_gemm.
+ * Contract: 1 <= M <= 2^24, 64 <= N <= 2^19, N % 8 == 0, K % 256 == 0, 256 <= K <= 2^20,
+ *           1 <= G <= 4096; A, B, sfa, sfb, C 16-byte aligned; alpha, m_indices 4-byte aligned.
+ */
+bsg_status bsg_nvfp4_gemm(const void* A, const void* B, const void* sfa, const void* sfb, const float* alpha,
+                          const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G,
+                          bsg_stream_t stream);
+
+/* Description of the last failure on the calling thread ("" if none).  The string stays valid until
+ * the next bsg_* call on the same thread. */
+const char* bsg_last_error(void);
+
+/*
+ * Device-side status: every bounded wait in the kernels (pipeline barriers, TMA arrivals) gives up
+ * after a time limit instead of hanging, records where it stopped in a device status word and makes
+ * the kernel return.  This call synchronises `stream`, reads and clears the word of the current
+ * device, and returns BSG_OK or BSG_ERR_DEVICE_TIMEOUT (details in bsg_last_error()).
+ */
+bsg_status bsg_get_device_status(bsg_stream_t stream);
+
+/*
+ * Wait limit of the kernels' bounded waits, in nanoseconds (default 2e9 = 2 s; applies to launches
+ * made after the call, from any thread).  Returns the previous value.  0 restores the default.
+ */
+uint64_t bsg_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * Tile / grid chooser (the tactic ranking of the page "[flashinfer] FlashInfer의 FP4 GEMM 최적화:
+ * 휴리스틱 개선과 Autotuning 효율화", section 2).  Tactic ids are small integers; bsg_tactic_name()
+ * describes one.  bsg_choose_tactic() returns the best-scored tactic for a shape (kind 0 = FP8,
+ * 1 = NVFP4; m_rows = routed rows, segments = an estimate of the number of per-expert window
+ * segments, sm_count = SMs on the device) or a negative bsg_status.  bsg_set_tactic() forces a tactic
+ * for later calls of that kind (-1 = let the chooser decide); the environment variable BSG_TACTIC
+ * does the same at load time.
+ */
+int bsg_num_tactics(int kind);
+const char* bsg_tactic_name(int kind, int tactic);
+int bsg_choose_tactic(int kind, int64_t m_rows, int64_t segments, int64_t N, int64_t K, int sm_count);
+double bsg_tactic_score(int kind, int tactic, int64_t m_rows, int64_t segments, int64_t N, int64_t K,
+                        int sm_count);
+bsg_status bsg_set_tactic(int kind, int tactic);
+
+/*
+ * Upper bound on the persistent grid of later calls of one kind (0 = FP8, 1 = NVFP4); 0 restores the
+ * default (one CTA per SM, fewer when there are fewer work units).  Any value >= 1 gives the same
+ * results, only slower: each CTA then walks more work units through the same pipelines.
+ */
+bsg_status bsg_set_max_ctas(int kind, int max_ctas);
+
+/*
+ * Test-only fault injection, for checking the bounded waits without faulting a GPU.  mode 0: off.
+ * mode 1: in later launches the scheduler warp hands out no work, so the other warps' bounded waits
+ * on the work queue expire after the wait limit; those launches issue no memory operation, release
+ * their tensor memory and return, and bsg_get_device_status() then reports BSG_ERR_DEVICE_TIMEOUT.
+ */
+bsg_status bsg_debug_set_fault(int mode);
+
+/* Library version string. */
+const char* bsg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSG_H_ */

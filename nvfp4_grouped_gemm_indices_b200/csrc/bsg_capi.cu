@@ -1,0 +1,351 @@
+// bsg_capi.cu -- the extern "C" boundary of libbsg.so: argument checks, TMA descriptor encoding,
+// tactic choice and kernel launch.  Declarations and the full contract are in include/bsg.h.
+//
+// The argument checks follow the host binding of the page "[flashinfer] FlashInfer FP8 GEMM 최적화:
+// 윈도우 세그먼트 KG1 프로그램으로 GPU 성능 극대화", section 1 (rank and unit-inner-stride checks,
+// K % 128, 16-byte strides and base addresses, boxes larger than an extent only on axes that may run
+// past the end, descriptive messages) and the launch contract of its section 2 (1 <= M <= 2^24,
+// 64 <= N <= 2^19).  Nothing is launched when a check fails.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/bsg.h"
+#include "bsg_chooser.h"
+#include "bsg_fp8.cuh"
+#include "bsg_nvfp4.cuh"
+
+#define BSG_VERSION_STRING "bsg 0.1.0 (sm_100a)"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+bsg_status fail(bsg_status code, const char* fmt, ...) {
+  char buf[1024];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+__device__ bsg::DeviceStatus g_device_status;
+
+uint64_t g_timeout_ns = 2000000000ull;
+int g_debug_fault = 0;
+std::mutex g_mu;
+
+constexpr int kMaxDevices = 64;
+struct DeviceState {
+  bool ready = false;
+  int sm_count = 0;
+  bsg::DeviceStatus* status = nullptr;
+  bool fp8_attr = false;
+  bool nvfp4_attr = false;
+};
+DeviceState g_dev[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+bsg_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(BSG_ERR_CUDA, "%s failed: %s (%d)", what, cudaGetErrorString(e), static_cast<int>(e));
+}
+
+// Per-device set-up (once per device, with that device current): SM count, the device address of
+// the status word, the kernels' shared-memory attribute.
+bsg_status device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(BSG_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    int major = 0, minor = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute(major)");
+    if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute(minor)");
+    if (major != 10 || minor != 0)
+      return fail(BSG_ERR_CUDA, "device %d is sm_%d%d; this library is built for sm_100a (B200) only", dev, major,
+                  minor);
+    if ((e = cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+    void* addr = nullptr;
+    if ((e = cudaGetSymbolAddress(&addr, g_device_status)) != cudaSuccess)
+      return cuda_fail(e, "cudaGetSymbolAddress(status word)");
+    st.status = static_cast<bsg::DeviceStatus*>(addr);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+      if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+        return fail(BSG_ERR_CUDA, "cannot resolve cuTensorMapEncodeTiled from the driver");
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    st.ready = true;
+  }
+  *out = &st;
+  return BSG_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Encodes a tiled descriptor after the same checks as the page's binding: extents >= box unless the
+// axis may run past the end, strides multiples of 16 bytes, 16-byte aligned base.
+bsg_status encode(CUtensorMap* map, const char* name, const void* base, int rank, const uint64_t* dims,
+                  const uint64_t* strides_bytes, const uint32_t* box, const bool* allow_oob,
+                  CUtensorMapSwizzle swz) {
+  if (!aligned(base, 16)) return fail(BSG_ERR_ALIGNMENT, "operand %s: base address must be 16-byte aligned", name);
+  for (int i = 0; i < rank; ++i) {
+    if (dims[i] == 0 || dims[i] > (1ull << 32))
+      return fail(BSG_ERR_UNSUPPORTED_SHAPE, "operand %s: extent %llu on axis %d outside [1, 2^32]", name,
+                  static_cast<unsigned long long>(dims[i]), i);
+    if (!allow_oob[i] && box[i] > dims[i])
+      return fail(BSG_ERR_UNSUPPORTED_SHAPE,
+                  "operand %s: axis %d (0 = innermost) has a TMA box of %u elements but the extent is %llu; "
+                  "this axis may not run past its end",
+                  name, i, box[i], static_cast<unsigned long long>(dims[i]));
+  }
+  for (int i = 0; i + 1 < rank; ++i) {
+    if (strides_bytes[i] % 16 != 0 || strides_bytes[i] >= (1ull << 40))
+      return fail(BSG_ERR_ALIGNMENT, "operand %s: stride %llu bytes (axis %d) must be a multiple of 16 below 2^40",
+                  name, static_cast<unsigned long long>(strides_bytes[i]), i + 1);
+  }
+  cuuint64_t gdim[5], gstr[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) gstr[i] = strides_bytes[i];
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<cuuint32_t>(rank), const_cast<void*>(base),
+                        gdim, gstr, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(BSG_ERR_CUDA, "cuTensorMapEncodeTiled of %s failed (CUresult %d)", name, (int)r);
+  return BSG_OK;
+}
+
+bsg_status check_common(const void* A, const void* B, const int32_t* m_indices, const void* C, int64_t M, int64_t N,
+                        int64_t K, int64_t G) {
+  if (!A || !B || !C) return fail(BSG_ERR_INVALID_ARG, "A, B and C must be non-null device pointers");
+  if (G < 1 || G > 4096) return fail(BSG_ERR_UNSUPPORTED_SHAPE, "G = %lld outside [1, 4096]", (long long)G);
+  if (!m_indices && G != 1)
+    return fail(BSG_ERR_INVALID_ARG, "m_indices may be NULL only when G == 1 (G = %lld)", (long long)G);
+  if (M < 1 || M > (1ll << 24))
+    return fail(BSG_ERR_UNSUPPORTED_SHAPE, "M = %lld outside the launch contract 1 <= M <= 2^24", (long long)M);
+  if (N < 64 || N > (1ll << 19))
+    return fail(BSG_ERR_UNSUPPORTED_SHAPE, "N = %lld outside the launch contract 64 <= N <= 2^19", (long long)N);
+  if (N % 8 != 0)
+    return fail(BSG_ERR_ALIGNMENT, "N = %lld must be a multiple of 8 (16-byte BF16 output rows)", (long long)N);
+  if (K > (1ll << 20)) return fail(BSG_ERR_UNSUPPORTED_SHAPE, "K = %lld above 2^20", (long long)K);
+  if (!aligned(C, 16)) return fail(BSG_ERR_ALIGNMENT, "C must be 16-byte aligned");
+  if (m_indices && !aligned(m_indices, 4)) return fail(BSG_ERR_ALIGNMENT, "m_indices must be 4-byte aligned");
+  return BSG_OK;
+}
+
+int grid_for(int sm_count, int64_t M, int64_t N, int64_t G, int bn) {
+  const int64_t n_tiles = (N + bn - 1) / bn;
+  const int64_t windows = (M + 127) / 128;
+  const int64_t segs = windows + (G < M ? G : M);  // sorted routing: at most one extra segment per expert
+  const int64_t units = n_tiles * segs;
+  return static_cast<int>(units < sm_count ? units : sm_count);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* bsg_version(void) { return BSG_VERSION_STRING; }
+
+const char* bsg_last_error(void) { return g_last_error.c_str(); }
+
+uint64_t bsg_set_wait_timeout_ns(uint64_t ns) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  uint64_t prev = g_timeout_ns;
+  g_timeout_ns = ns ? ns : 2000000000ull;
+  return prev;
+}
+
+static uint64_t current_timeout() {
+  std::lock_guard<std::mutex> lock(g_mu);
+  return g_timeout_ns;
+}
+
+static int current_fault() {
+  std::lock_guard<std::mutex> lock(g_mu);
+  return g_debug_fault;
+}
+
+bsg_status bsg_debug_set_fault(int mode) {
+  if (mode < 0 || mode > bsg::kDebugWithholdSchedule) return fail(BSG_ERR_INVALID_ARG, "unknown fault mode %d", mode);
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_debug_fault = mode;
+  return BSG_OK;
+}
+
+bsg_status bsg_fp8_grouped_gemm(const void* A, const void* B, const float* a_scale, const float* b_scale,
+                                const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G,
+                                bsg_stream_t stream) {
+  g_last_error.clear();
+  bsg_status st = check_common(A, B, m_indices, C, M, N, K, G);
+  if (st != BSG_OK) return st;
+  if (!a_scale || !b_scale) return fail(BSG_ERR_INVALID_ARG, "a_scale and b_scale must be non-null");
+  if (K < 128 || K % 128 != 0)
+    return fail(BSG_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 128 (one FP32 scale per 128)",
+                (long long)K);
+  if (!aligned(A, 16) || !aligned(B, 16)) return fail(BSG_ERR_ALIGNMENT, "A and B must be 16-byte aligned");
+  if (!aligned(a_scale, 4) || !aligned(b_scale, 4))
+    return fail(BSG_ERR_ALIGNMENT, "a_scale and b_scale must be 4-byte aligned");
+  DeviceState* dev = nullptr;
+  if ((st = device_state(&dev)) != BSG_OK) return st;
+
+  bsg::Fp8Params p;
+  memset(&p, 0, sizeof(p));
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+    const uint64_t str[1] = {static_cast<uint64_t>(K)};
+    const uint32_t box[2] = {128u, 128u};
+    const bool oob[2] = {false, true};  // the last window may run past M: zero-filled, rows masked
+    if ((st = encode(&p.tmA, "A", A, 2, dims, str, box, oob, CU_TENSOR_MAP_SWIZZLE_128B)) != BSG_OK) return st;
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), static_cast<uint64_t>(G)};
+    const uint64_t str[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N) * static_cast<uint64_t>(K)};
+    const uint32_t box[3] = {128u, static_cast<uint32_t>(bsg::fp8::BN), 1u};
+    const bool oob[3] = {false, true, false};  // an N tail tile is zero-filled, columns masked
+    if ((st = encode(&p.tmB, "B", B, 3, dims, str, box, oob, CU_TENSOR_MAP_SWIZZLE_128B)) != BSG_OK) return st;
+  }
+  p.a_scale = a_scale;
+  p.b_scale = b_scale;
+  p.m_indices = m_indices;
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.G = static_cast<int>(G);
+  p.timeout_ns = current_timeout();
+  p.status = dev->status;
+  p.debug_mode = current_fault();
+
+  cudaError_t e;
+  if (!dev->fp8_attr) {
+    e = cudaFuncSetAttribute(bsg::fp8::kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bsg::fp8::SMEM_BYTES));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fp8 kernel smem)");
+    dev->fp8_attr = true;
+  }
+  const int grid = bsg_forced_grid(0, grid_for(dev->sm_count, M, N, G, bsg::fp8::BN));
+  bsg::fp8::kernel<<<grid, bsg::fp8::THREADS, bsg::fp8::SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the fp8 grouped kernel");
+  return BSG_OK;
+}
+
+bsg_status bsg_nvfp4_gemm(const void* A, const void* B, const void* sfa, const void* sfb, const float* alpha,
+                          const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G,
+                          bsg_stream_t stream) {
+  g_last_error.clear();
+  bsg_status st = check_common(A, B, m_indices, C, M, N, K, G);
+  if (st != BSG_OK) return st;
+  if (!sfa || !sfb || !alpha) return fail(BSG_ERR_INVALID_ARG, "sfa, sfb and alpha must be non-null");
+  if (K < 256 || K % 256 != 0)
+    return fail(BSG_ERR_UNSUPPORTED_SHAPE,
+                "K = %lld must be a positive multiple of 256 (16-byte rows of packed codes and of scale bytes)",
+                (long long)K);
+  if (!aligned(alpha, 4)) return fail(BSG_ERR_ALIGNMENT, "alpha must be 4-byte aligned");
+  DeviceState* dev = nullptr;
+  if ((st = device_state(&dev)) != BSG_OK) return st;
+
+  bsg::Nvfp4Params p;
+  memset(&p, 0, sizeof(p));
+  const uint64_t Kb = static_cast<uint64_t>(K) / 2;   // packed bytes per row
+  const uint64_t Ks = static_cast<uint64_t>(K) / 16;  // scale bytes per row
+  {
+    const uint64_t dims[2] = {Kb, static_cast<uint64_t>(M)};
+    const uint64_t str[1] = {Kb};
+    const uint32_t box[2] = {128u, 128u};
+    const bool oob[2] = {false, true};
+    if ((st = encode(&p.tmA, "A", A, 2, dims, str, box, oob, CU_TENSOR_MAP_SWIZZLE_128B)) != BSG_OK) return st;
+  }
+  {
+    const uint64_t dims[3] = {Kb, static_cast<uint64_t>(N), static_cast<uint64_t>(G)};
+    const uint64_t str[2] = {Kb, static_cast<uint64_t>(N) * Kb};
+    const uint32_t box[3] = {128u, static_cast<uint32_t>(bsg::nvfp4::BN), 1u};
+    const bool oob[3] = {false, true, false};
+    if ((st = encode(&p.tmB, "B", B, 3, dims, str, box, oob, CU_TENSOR_MAP_SWIZZLE_128B)) != BSG_OK) return st;
+  }
+  {
+    const uint64_t dims[2] = {Ks, static_cast<uint64_t>(M)};
+    const uint64_t str[1] = {Ks};
+    const uint32_t box[2] = {16u, 128u};
+    const bool oob[2] = {false, true};
+    if ((st = encode(&p.tmSFA, "sfa", sfa, 2, dims, str, box, oob, CU_TENSOR_MAP_SWIZZLE_NONE)) != BSG_OK) return st;
+  }
+  {
+    const uint64_t dims[3] = {Ks, static_cast<uint64_t>(N), static_cast<uint64_t>(G)};
+    const uint64_t str[2] = {Ks, static_cast<uint64_t>(N) * Ks};
+    const uint32_t box[3] = {16u, static_cast<uint32_t>(bsg::nvfp4::BN), 1u};
+    const bool oob[3] = {false, true, false};
+    if ((st = encode(&p.tmSFB, "sfb", sfb, 3, dims, str, box, oob, CU_TENSOR_MAP_SWIZZLE_NONE)) != BSG_OK) return st;
+  }
+  p.alpha = alpha;
+  p.m_indices = m_indices;
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.G = static_cast<int>(G);
+  p.timeout_ns = current_timeout();
+  p.status = dev->status;
+  p.debug_mode = current_fault();
+
+  cudaError_t e;
+  if (!dev->nvfp4_attr) {
+    e = cudaFuncSetAttribute(bsg::nvfp4::kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bsg::nvfp4::SMEM_BYTES));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(nvfp4 kernel smem)");
+    dev->nvfp4_attr = true;
+  }
+  const int grid = bsg_forced_grid(1, grid_for(dev->sm_count, M, N, G, bsg::nvfp4::BN));
+  bsg::nvfp4::kernel<<<grid, bsg::nvfp4::THREADS, bsg::nvfp4::SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(
+      p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the nvfp4 kernel");
+  return BSG_OK;
+}
+
+bsg_status bsg_get_device_status(bsg_stream_t stream) {
+  g_last_error.clear();
+  DeviceState* dev = nullptr;
+  bsg_status st = device_state(&dev);
+  if (st != BSG_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  bsg::DeviceStatus hs;
+  e = cudaMemcpy(&hs, dev->status, sizeof(hs), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  if (hs.word == 0) return BSG_OK;
+  bsg::DeviceStatus zero = {0u, 0u};
+  e = cudaMemcpy(dev->status, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+  return fail(BSG_ERR_DEVICE_TIMEOUT,
+              "a kernel gave up a bounded wait: site %u, stage %u, block %u, parity %u (status word 0x%08x)",
+              (hs.word >> 20) & 0xFu, (hs.word >> 12) & 0xFFu, hs.word & 0xFFFu, hs.detail, hs.word);
+}
+
+}  // extern "C"

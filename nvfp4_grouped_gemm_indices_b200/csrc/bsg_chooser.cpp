@@ -1,0 +1,154 @@
+// bsg_chooser.cpp -- the tile / cluster chooser.
+//
+// Score of a tactic (the ranking of the page "[flashinfer] FlashInfer의 FP4 GEMM 최적화: 휴리스틱
+// 개선과 Autotuning 효율화", section 2):
+//     score = m_eff * n_eff * throughput / (num_waves * tile_n)
+//     score *= 1.05            if the tactic issues 2-CTA (cta_group::2) MMAs
+//     score *= 0.95^(log2 cga_n)   for a cluster of cga_n CTAs along N (multicast)
+// The page names but does not define m_eff, n_eff, throughput and num_waves.  Readings used here:
+//     m_eff      = useful rows / rows computed = M_routed / (segments * tile_m)   (window segments are
+//                  the row tiles of this library, so the padding they waste is what m_eff measures)
+//     n_eff      = N / (ceil(N / tile_n) * tile_n)
+//     num_waves  = ceil(units / (sm_count / cluster_size)), units = segments * ceil(N / tile_n)
+//     throughput = the tile's relative tensor-core rate (1.0 for the full 128 x 256 issue shape,
+//                  proportionally less for narrower N tiles that leave the pipe shared-memory bound)
+// The exhaustive sweep over all tactics (bench.py --sweep) is what validates the ranking.
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+
+#include "../../include/bsg.h"
+#include "bsg_chooser.h"
+
+namespace {
+
+struct Tactic {
+  const char* name;
+  int tile_m;
+  int tile_n;
+  int cta_group;
+  int cga_n;
+  double throughput;
+};
+
+// FP8 and NVFP4 tactic tables (kind 0 and 1).  Only tactics that exist as kernels are listed.
+const Tactic kFp8[] = {
+    {"fp8_1sm_m128_n256_s4", 128, 256, 1, 1, 1.0},
+};
+const Tactic kNvfp4[] = {
+    {"nvfp4_1sm_m128_n256_s4", 128, 256, 1, 1, 1.0},
+};
+
+const Tactic* table(int kind, int* n) {
+  if (kind == 0) {
+    *n = static_cast<int>(sizeof(kFp8) / sizeof(kFp8[0]));
+    return kFp8;
+  }
+  if (kind == 1) {
+    *n = static_cast<int>(sizeof(kNvfp4) / sizeof(kNvfp4[0]));
+    return kNvfp4;
+  }
+  *n = 0;
+  return nullptr;
+}
+
+std::mutex g_mu;
+int g_forced_tactic[2] = {-1, -1};
+int g_max_ctas[2] = {0, 0};
+bool g_env_read = false;
+
+void read_env() {
+  if (g_env_read) return;
+  g_env_read = true;
+  if (const char* t = std::getenv("BSG_TACTIC")) {
+    int v = std::atoi(t);
+    g_forced_tactic[0] = g_forced_tactic[1] = v;
+  }
+}
+
+}  // namespace
+
+int bsg_forced_grid(int kind, int grid) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (kind < 0 || kind > 1) return grid;
+  int cap = g_max_ctas[kind];
+  if (cap > 0 && cap < grid) return cap;
+  return grid;
+}
+
+extern "C" {
+
+int bsg_num_tactics(int kind) {
+  int n = 0;
+  table(kind, &n);
+  return n;
+}
+
+const char* bsg_tactic_name(int kind, int tactic) {
+  int n = 0;
+  const Tactic* t = table(kind, &n);
+  if (!t || tactic < 0 || tactic >= n) return "";
+  return t[tactic].name;
+}
+
+double bsg_tactic_score(int kind, int tactic, int64_t m_rows, int64_t segments, int64_t N, int64_t K, int sm_count) {
+  (void)K;
+  int n = 0;
+  const Tactic* tt = table(kind, &n);
+  if (!tt || tactic < 0 || tactic >= n || m_rows <= 0 || segments <= 0 || N <= 0 || sm_count <= 0) return 0.0;
+  const Tactic& t = tt[tactic];
+  const double tiles_n = std::ceil(static_cast<double>(N) / t.tile_n);
+  const double m_eff = static_cast<double>(m_rows) / (static_cast<double>(segments) * t.tile_m);
+  const double n_eff = static_cast<double>(N) / (tiles_n * t.tile_n);
+  const int cluster = t.cta_group * t.cga_n;
+  const double units = static_cast<double>(segments) * tiles_n / t.cta_group;
+  const double slots = std::floor(static_cast<double>(sm_count) / cluster);
+  const double waves = std::ceil(units / (slots > 0 ? slots : 1.0));
+  double score = m_eff * n_eff * t.throughput / (waves * t.tile_n);
+  if (t.cta_group == 2) score *= 1.05;
+  int bits = 0;
+  for (int v = t.cga_n; v > 1; v >>= 1) ++bits;
+  score *= std::pow(0.95, bits);
+  return score;
+}
+
+int bsg_choose_tactic(int kind, int64_t m_rows, int64_t segments, int64_t N, int64_t K, int sm_count) {
+  int n = 0;
+  if (!table(kind, &n)) return BSG_ERR_INVALID_ARG;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    read_env();
+    int f = g_forced_tactic[kind];
+    if (f >= 0 && f < n) return f;
+  }
+  int best = 0;
+  double best_score = -1.0;
+  for (int i = 0; i < n; ++i) {
+    double s = bsg_tactic_score(kind, i, m_rows, segments, N, K, sm_count);
+    if (s > best_score) {
+      best_score = s;
+      best = i;
+    }
+  }
+  return best;
+}
+
+bsg_status bsg_set_tactic(int kind, int tactic) {
+  int n = 0;
+  if (!table(kind, &n)) return BSG_ERR_INVALID_ARG;
+  if (tactic >= n) return BSG_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  read_env();
+  g_forced_tactic[kind] = tactic < 0 ? -1 : tactic;
+  return BSG_OK;
+}
+
+bsg_status bsg_set_max_ctas(int kind, int max_ctas) {
+  if (kind < 0 || kind > 1 || max_ctas < 0) return BSG_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_max_ctas[kind] = max_ctas;
+  return BSG_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,145 @@
+"""CPU-side checks of the C ABI: the library loads without a GPU, exports every function
+include/bsg.h declares, rejects bad arguments on the host (launching nothing), and its chooser
+ranks tactics by the page's score."""
+import os
+import re
+
+import pytest
+
+import nvfp4_grouped_gemm_indices_b200 as bsg
+from nvfp4_grouped_gemm_indices_b200 import build as bsg_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    bsg_build.build()
+    return bsg.load()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "bsg.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bsg_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    assert "bsg_fp8_grouped_gemm" in names and "bsg_nvfp4_gemm" in names
+    assert sorted(bsg.EXPORTED) == names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version(lib):
+    assert "sm_100a" in bsg.bsg_version()
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null "device" address; never dereferenced by the host checks
+
+
+def fp8_args(**kw):
+    a = dict(A=FAKE, B=FAKE, a_scale=FAKE, b_scale=FAKE, m_indices=FAKE, C=FAKE, M=512, N=256, K=512, G=4)
+    a.update(kw)
+    return a
+
+
+def nvfp4_args(**kw):
+    a = dict(A=FAKE, B=FAKE, sfa=FAKE, sfb=FAKE, alpha=FAKE, m_indices=FAKE, C=FAKE, M=512, N=256, K=512, G=4)
+    a.update(kw)
+    return a
+
+
+@pytest.mark.parametrize("kw,status,needle", [
+    (dict(A=0), bsg.BSG_ERR_INVALID_ARG, "non-null"),
+    (dict(C=0), bsg.BSG_ERR_INVALID_ARG, "non-null"),
+    (dict(a_scale=0), bsg.BSG_ERR_INVALID_ARG, "a_scale"),
+    (dict(m_indices=0), bsg.BSG_ERR_INVALID_ARG, "G == 1"),
+    (dict(M=0), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "M = 0"),
+    (dict(M=(1 << 24) + 1), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "2^24"),
+    (dict(N=32), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "64 <= N"),
+    (dict(N=(1 << 19) + 8), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "2^19"),
+    (dict(N=100), bsg.BSG_ERR_ALIGNMENT, "multiple of 8"),
+    (dict(K=200), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "multiple of 128"),
+    (dict(K=0), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "multiple of 128"),
+    (dict(G=0), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "G = 0"),
+    (dict(G=5000), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "4096"),
+    (dict(A=FAKE + 8), bsg.BSG_ERR_ALIGNMENT, "16-byte"),
+    (dict(C=FAKE + 4), bsg.BSG_ERR_ALIGNMENT, "16-byte"),
+    (dict(a_scale=FAKE + 2), bsg.BSG_ERR_ALIGNMENT, "4-byte"),
+    (dict(m_indices=FAKE + 1), bsg.BSG_ERR_ALIGNMENT, "4-byte"),
+])
+def test_fp8_argument_errors(lib, kw, status, needle):
+    with pytest.raises(bsg.BsgError) as ei:
+        bsg.bsg_fp8_grouped_gemm(**fp8_args(**kw), stream=0)
+    assert ei.value.status == status
+    assert needle in str(ei.value)
+
+
+@pytest.mark.parametrize("kw,status,needle", [
+    (dict(sfa=0), bsg.BSG_ERR_INVALID_ARG, "sfa"),
+    (dict(alpha=0), bsg.BSG_ERR_INVALID_ARG, "alpha"),
+    (dict(K=128), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "multiple of 256"),
+    (dict(K=384), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "multiple of 256"),
+    (dict(alpha=FAKE + 2), bsg.BSG_ERR_ALIGNMENT, "alpha"),
+    (dict(M=-3), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "M = -3"),
+])
+def test_nvfp4_argument_errors(lib, kw, status, needle):
+    with pytest.raises(bsg.BsgError) as ei:
+        bsg.bsg_nvfp4_gemm(**nvfp4_args(**kw), stream=0)
+    assert ei.value.status == status
+    assert needle in str(ei.value)
+
+
+def test_valid_call_without_gpu_reports_cuda_error(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(bsg.BsgError) as ei:
+        bsg.bsg_fp8_grouped_gemm(**fp8_args(), stream=0)
+    assert ei.value.status == bsg.BSG_ERR_CUDA
+
+
+def test_null_routing_allowed_for_single_expert(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(bsg.BsgError) as ei:  # passes the host checks, then finds no device
+        bsg.bsg_nvfp4_gemm(**nvfp4_args(m_indices=0, G=1), stream=0)
+    assert ei.value.status == bsg.BSG_ERR_CUDA
+
+
+def test_timeout_setter_roundtrip(lib):
+    prev = bsg.bsg_set_wait_timeout_ns(123456789)
+    assert bsg.bsg_set_wait_timeout_ns(0) == 123456789
+    assert bsg.bsg_set_wait_timeout_ns(prev) == 2000000000
+
+
+def test_chooser_score_follows_the_page_formula(lib):
+    for kind in (0, 1):
+        n = bsg.bsg_num_tactics(kind)
+        assert n >= 1
+        for t in range(n):
+            assert bsg.bsg_tactic_name(kind, t)
+            s = bsg.bsg_tactic_score(kind, t, 8192, 71, 4096, 7168, 148)
+            assert s > 0
+        best = bsg.bsg_choose_tactic(kind, 8192, 71, 4096, 7168, 148)
+        scores = [bsg.bsg_tactic_score(kind, t, 8192, 71, 4096, 7168, 148) for t in range(n)]
+        assert best == max(range(n), key=lambda t: scores[t])
+    # a single-tactic check of the formula: 64 full windows, N = 4096, tile 128 x 256, 148 SMs
+    s = bsg.bsg_tactic_score(0, 0, 8192, 64, 4096, 7168, 148)
+    waves = -(-(64 * 16) // 148)
+    assert abs(s - 1.0 * 1.0 * 1.0 / (waves * 256)) < 1e-15
+    assert bsg.bsg_tactic_score(0, 99, 1, 1, 64, 128, 148) == 0.0
+
+
+def test_set_max_ctas_validation(lib):
+    with pytest.raises(bsg.BsgError):
+        bsg.bsg_set_max_ctas(2, 1)
+    with pytest.raises(bsg.BsgError):
+        bsg.bsg_set_max_ctas(0, -1)
+    bsg.bsg_set_max_ctas(0, 0)
