@@ -1,0 +1,509 @@
+#!/usr/bin/env python
+"""Benchmark of the block-scaled grouped GEMM on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl bsg|reference] [--config I]
+                    [--no-also] [--cpu-seconds S]
+
+One step = one launch of the whole hot path (window scheduling, TMA loads, scale handling, tcgen05
+MMAs, BF16 epilogue -- all inside one kernel) over one batch of synthetic input.  The headline
+workload is the FP8 grouped MoE prefill (G=8, M=8192, N=4096, K=7168); `--config` picks another of
+the five workloads.  The timed region is K back-to-back launches bracketed by a barrier and a device
+synchronisation, timed with CUDA events on the launching stream, max over ranks.  Inputs are larger
+than the 126 MB L2 for the headline workload (stated in the JSON `config`); smaller workloads flush
+L2 between launches outside the per-launch events.
+
+Rank 0 prints ONE JSON line (metric, value = whole-job TFLOPS, roofline of the kernel, the oracle's
+CPU throughput on a bounded sample, the end-to-end number through host buffers, clocks sampled
+during the timed region).  `--impl reference` times the fp64 CPU oracle on the same workload instead
+(rank 0 only).  Under torchrun each rank runs its own copy of the workload on its own GPU (weak
+scaling, no data-path collective: the op needs no exchange step).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "grouped block-scaled GEMM TFLOPS (FP8 & NVFP4) + % of B200 roofline"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# nominal dense ratios to bf16 (2.25 PF): fp8 4.5 PF, fp4 9 PF
+DTYPE_RATIO = {"fp8": 2.0, "nvfp4": 4.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["bsg", "reference"], default="bsg")
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--no-also", action="store_true", help="skip the other workloads' kernel numbers")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- distributed helpers
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(backend, timeout_s=120):
+    import datetime
+
+    import torch.distributed as dist
+    ws, rank, _ = dist_env()
+    if ws > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return ws, rank
+
+
+def reduce_max(value, device=None):
+    """Max of a float over ranks (the slowest rank sets the job time); identity when not distributed."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def job_value(per_rank_flops, max_seconds, world):
+    """Whole-job throughput in TFLOPS: every rank processes its own (identical-size) batch."""
+    return world * per_rank_flops / max_seconds / 1e12
+
+
+# ----------------------------------------------------------------------------- peaks / clocks
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def visible_gpu_index(local_rank):
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if cvd:
+        ids = [x.strip() for x in cvd.split(",") if x.strip()]
+        if local_rank < len(ids) and ids[local_rank].isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
+# ----------------------------------------------------------------------------- kernel source hash
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "nvfp4_grouped_gemm_indices_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per launch from a committed ncu capture, if taken on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload_name)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- our arm
+
+
+class Runner:
+    def __init__(self, w):
+        import torch
+
+        import nvfp4_grouped_gemm_indices_b200 as bsg
+        self.bsg = bsg
+        self.w = w
+        dev = lambda x: None if x is None else torch.from_numpy(np.ascontiguousarray(x)).cuda()
+        self.A, self.B, self.idx = dev(w.A), dev(w.B), dev(w.m_indices)
+        if w.kind == "fp8":
+            self.s1, self.s2, self.s3 = dev(w.a_scale), dev(w.b_scale), None
+        else:
+            self.s1, self.s2, self.s3 = dev(w.sfa), dev(w.sfb), dev(w.alpha)
+        self.C = torch.zeros((w.M, w.N), dtype=torch.bfloat16, device="cuda")
+
+    def launch(self, stream, A=None, B=None, s1=None, s2=None, s3=None, idx=None, C=None):
+        w = self.w
+        A = self.A if A is None else A
+        B = self.B if B is None else B
+        s1 = self.s1 if s1 is None else s1
+        s2 = self.s2 if s2 is None else s2
+        s3 = self.s3 if s3 is None else s3
+        idx = self.idx if idx is None else idx
+        C = self.C if C is None else C
+        if w.kind == "fp8":
+            self.bsg.bsg_fp8_grouped_gemm(A, B, s1, s2, idx, C, w.M, w.N, w.K, w.G, stream)
+        else:
+            self.bsg.bsg_nvfp4_gemm(A, B, s1, s2, s3, idx, C, w.M, w.N, w.K, w.G, stream)
+
+
+def time_kernel(runner, steps, warmup, flush=None):
+    """K back-to-back launches between synchronisations; returns (total seconds, mean per-launch
+    seconds from per-launch event pairs on the launching stream)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        runner.launch(stream.cuda_stream)
+    torch.cuda.synchronize()
+    runner.bsg.bsg_get_device_status()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(steps):
+        if flush is not None:
+            flush()
+        starts[i].record(stream)
+        runner.launch(stream.cuda_stream)
+        ends[i].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    runner.bsg.bsg_get_device_status()
+    total = t0.elapsed_time(t1) / 1e3
+    per = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / steps / 1e3
+    return total, per
+
+
+def time_e2e(runner, steps):
+    """Host buffers in pinned memory: every step copies all operands host->device, runs the kernel
+    through the C ABI and copies C back; timed with CUDA events on the stream."""
+    import torch
+    w = runner.w
+    host = {}
+    for name in ("A", "B", "s1", "s2", "s3", "idx"):
+        t = getattr(runner, name)
+        if t is not None:
+            host[name] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            host[name].copy_(t.cpu())
+    dev = {k: torch.empty_like(getattr(runner, k)) for k in host}
+    Cdev = torch.empty_like(runner.C)
+    Chost = torch.empty(runner.C.shape, dtype=runner.C.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = Chost.numel() * Chost.element_size()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for k, t in host.items():
+            dev[k].copy_(t, non_blocking=True)
+        runner.launch(stream.cuda_stream, C=Cdev, **dev)
+        Chost.copy_(Cdev, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    return e0.elapsed_time(e1) / 1e3 / steps, h2d, d2h
+
+
+def make_flush():
+    import torch
+    buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device="cuda")
+
+    def flush():
+        buf.fill_(1)
+    return flush
+
+
+def roofline(w, per_launch_s, peaks, peak_src, sustained=False):
+    bf16 = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    tensor_peak = bf16 * DTYPE_RATIO[w.kind]
+    hbm = peaks["hbm_gbs"]
+    flops = w.flops
+    nbytes = w.algorithmic_bytes()
+    t_tensor = flops / (tensor_peak * 1e12)
+    t_hbm = nbytes / (hbm * 1e9)
+    traffic = recorded_traffic(w.name)
+    if t_hbm > t_tensor:
+        ach = nbytes / per_launch_s / 1e9
+        return {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(ach / hbm, 4), "traffic": traffic, "algorithmic_bytes": nbytes,
+                "peak_source": f"{peak_src} hbm_gbs (STREAM-style copy)"}
+    ach = flops / per_launch_s / 1e12
+    return {"bound": "tensor", "achieved": round(ach, 1), "peak": round(tensor_peak, 1), "unit": "TFLOP/s",
+            "frac": round(ach / tensor_peak, 4), "traffic": traffic, "algorithmic_bytes": nbytes,
+            "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} x {DTYPE_RATIO[w.kind]:g} "
+                           f"({w.kind} : bf16 nominal dense ratio)"}
+
+
+def cpu_baseline(w, seconds):
+    """The oracle as it stands, on the host's cores, over a bounded sample of the workload's rows
+    (all N columns each).  Returns (TFLOPS, cores, sample description)."""
+    import oracle
+    cores = oracle.max_threads()
+    routed = np.nonzero((w.m_indices >= 0) & (w.m_indices < w.G))[0] if w.m_indices is not None \
+        else np.arange(w.M)
+    rng = np.random.default_rng(1234)
+    # calibrate on one row per core
+    probe = rng.choice(routed, size=min(cores, len(routed)), replace=False)
+    t = time.perf_counter()
+    run_oracle(w, probe)
+    dt = time.perf_counter() - t
+    per_row = dt / len(probe)
+    n = int(max(len(probe), min(len(routed), seconds / max(per_row, 1e-9))))
+    n = max(cores, (n // cores) * cores) if n >= cores else n
+    rows = np.sort(rng.choice(routed, size=min(n, len(routed)), replace=False))
+    t = time.perf_counter()
+    run_oracle(w, rows)
+    dt = time.perf_counter() - t
+    flops = 2.0 * len(rows) * w.N * w.K
+    return flops / dt / 1e12, cores, f"{len(rows)} random routed rows x all {w.N} columns ({dt:.1f} s)"
+
+
+def run_oracle(w, rows, n_cols=None):
+    import oracle
+    if w.kind == "fp8":
+        if n_cols is None:
+            return oracle.fp8_grouped(w.A, w.B, w.a_scale, w.b_scale, w.m_indices, w.M, w.N, w.K, w.G, rows=rows)
+        return oracle.fp8_grouped(w.A, w.B[:, :n_cols], w.a_scale, w.b_scale[:, :(n_cols + 127) // 128],
+                                  w.m_indices, w.M, n_cols, w.K, w.G, rows=rows)
+    if n_cols is None:
+        return oracle.nvfp4(w.A, w.B, w.sfa, w.sfb, w.alpha, w.m_indices, w.M, w.N, w.K, w.G, rows=rows)
+    return oracle.nvfp4(w.A, w.B[:, :n_cols], w.sfa, w.sfb[:, :n_cols], w.alpha, w.m_indices, w.M, n_cols, w.K,
+                        w.G, rows=rows)
+
+
+def config_desc(w, cfg, flush):
+    d = {"workload": w.name, "config_index": cfg, "kind": w.kind, "M": w.M, "N": w.N, "K": w.K, "G": w.G,
+         "routed_rows": w.routed_rows, "active_experts": len(w.active_experts()),
+         "input_bytes": int(w.A.nbytes + w.B.nbytes + (w.m_indices.nbytes if w.m_indices is not None else 0)),
+         "parallelism": "replicas (one independent batch per GPU, no collective)"}
+    d["l2"] = ("L2 flushed (2x126 MB write) between launches, outside the per-launch events" if flush
+               else f"inputs {d['input_bytes'] / 1e6:.0f} MB > 126 MB L2, no flush")
+    return d
+
+
+def run_bsg(args):
+    import torch
+    ws, rank, local = dist_env()
+    if args.gpus != ws:
+        if ws == 1 and args.gpus > 1:
+            raise SystemExit("--gpus > 1 needs torchrun (one process per GPU)")
+    torch.cuda.set_device(local)
+    init_dist("nccl")
+    peaks, peak_src = load_peaks()
+
+    sampler = ClockSampler(visible_gpu_index(local))
+    from nvfp4_grouped_gemm_indices_b200 import workloads as W
+    w = W.config(args.config)
+    r = Runner(w)
+    flush = make_flush() if (w.A.nbytes + w.B.nbytes) < 2 * L2_BYTES else None
+    sampler.start()
+    total, per = time_kernel(r, args.steps, args.warmup, flush)
+    clocks = sampler.stop()
+    if flush is not None:
+        total = per * args.steps
+    total = reduce_max(total, device="cuda")
+    per = reduce_max(per, device="cuda")
+    ms_per_step = total / args.steps * 1e3
+    value = job_value(w.flops, total / args.steps, ws)
+
+    e2e_s, h2d, d2h = time_e2e(r, args.e2e_steps)
+    e2e_s = reduce_max(e2e_s, device="cuda")
+    e2e_value = job_value(w.flops, e2e_s, ws)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3xe4m3->f32 (fp32 per-128 scales), bf16 out" if w.kind == "fp8"
+        else "e2m1xe2m1 (ue4m3 per-16 scales)->f32, bf16 out",
+        "data": "synthetic (seeded; quantised N(0,1) activations, N(0,0.02) / N(0,1) weights)",
+        "config": config_desc(w, args.config, flush),
+        "roofline": roofline(w, per, peaks, peak_src),
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps,
+                "note": "all operands copied host->device from pinned memory and C copied back, every step"},
+    }
+    if ws == 1 and rank == 0:
+        tf, cores, sample = cpu_baseline(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample}
+        if not args.no_also:
+            also = {}
+            for cfg in (0, 2, 3, 4):
+                if cfg == args.config:
+                    continue
+                del r
+                torch.cuda.empty_cache()
+                wc = W.config(cfg)
+                r = Runner(wc)
+                fl = make_flush() if (wc.A.nbytes + wc.B.nbytes) < 2 * L2_BYTES else None
+                steps = max(20, min(args.steps, 200))
+                tot, pl = time_kernel(r, steps, max(3, args.warmup // 4), fl)
+                rf = roofline(wc, pl, peaks, peak_src)
+                also[wc.name] = {"tflops": round(wc.flops / pl / 1e12, 2), "us_per_launch": round(pl * 1e6, 2),
+                                 "roofline": rf, "l2": "flushed" if fl else "inputs > L2"}
+            line["also"] = also
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    from nvfp4_grouped_gemm_indices_b200 import workloads as W
+    import oracle
+    w = W.config(args.config)
+    cores = oracle.max_threads()
+    # per step: a bounded sample (rows x leading 128-column blocks) sized so that warmup + steps take
+    # about 90 s of CPU time in total
+    budget = 90.0 / max(1, args.steps + args.warmup)
+    routed = np.nonzero((w.m_indices >= 0) & (w.m_indices < w.G))[0] if w.m_indices is not None \
+        else np.arange(w.M)
+    rng = np.random.default_rng(99)
+    t = time.perf_counter()
+    run_oracle(w, routed[:cores], n_cols=128)
+    per_unit = (time.perf_counter() - t) / cores          # one row x 128 columns
+    units = max(1, int(budget / max(per_unit, 1e-9)))
+    rows_per_step = max(1, min(cores, units))
+    cols = int(min(w.N, max(128, 128 * (units // rows_per_step)))) // 128 * 128
+    for _ in range(args.warmup):
+        run_oracle(w, rng.choice(routed, rows_per_step, replace=False), n_cols=cols)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        run_oracle(w, rng.choice(routed, rows_per_step, replace=False), n_cols=cols)
+    dt = (time.perf_counter() - t) / args.steps
+    flops = 2.0 * rows_per_step * cols * w.K
+    value = flops / dt / 1e12
+    sample = f"per step {rows_per_step} random routed rows x the first {cols} columns of {w.name}"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (decoded operands)", "data": "synthetic",
+        "config": {"workload": w.name, "config_index": args.config, "M": w.M, "N": w.N, "K": w.K, "G": w.G},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_bsg(args)
+    try:
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
+            dist.destroy_process_group()
+    except Exception:
+        pass
+
+
+if __name__ == "__main__":
+    main()

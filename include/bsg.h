@@ -104,18 +104,17 @@ uint64_t bsg_set_wait_timeout_ns(uint64_t ns);
 
 /*
  * Tile / grid chooser (the tactic ranking of the page "[flashinfer] FlashInfer의 FP4 GEMM 최적화:
- * 휴리스틱 개선과 Autotuning 효율화", section 2).  Tactic ids are small integers; bsg_tactic_name()
- * describes one.  bsg_choose_tactic() returns the best-scored tactic for a shape (kind 0 = FP8,
- * 1 = NVFP4; m_rows = routed rows, segments = an estimate of the number of per-expert window
- * segments, sm_count = SMs on the device) or a negative bsg_status.  bsg_set_tactic() forces a tactic
- * for later calls of that kind (-1 = let the chooser decide); the environment variable BSG_TACTIC
- * does the same at load time.
+ * 휴리스틱 개선과 Autotuning 효율화", section 2).  Tactic ids are small integers per kind (0 = FP8,
+ * 1 = NVFP4); bsg_tactic_name() describes one.  bsg_tactic_score() is the page's score of a tactic
+ * for a problem size (M rows, N, K, G experts, sm_count SMs), with the work-unit counts estimated
+ * from the sizes alone; bsg_choose_tactic() returns the best-scored (or forced) tactic, or a
+ * negative bsg_status.  bsg_set_tactic() forces a tactic for later calls of that kind (-1 = let the
+ * chooser decide); the environment variable BSG_TACTIC does the same at load time.
  */
 int bsg_num_tactics(int kind);
 const char* bsg_tactic_name(int kind, int tactic);
-int bsg_choose_tactic(int kind, int64_t m_rows, int64_t segments, int64_t N, int64_t K, int sm_count);
-double bsg_tactic_score(int kind, int tactic, int64_t m_rows, int64_t segments, int64_t N, int64_t K,
-                        int sm_count);
+int bsg_choose_tactic(int kind, int64_t M, int64_t N, int64_t K, int64_t G, int sm_count);
+double bsg_tactic_score(int kind, int tactic, int64_t M, int64_t N, int64_t K, int64_t G, int sm_count);
 bsg_status bsg_set_tactic(int kind, int tactic);
 
 /*

@@ -154,15 +154,14 @@ def bsg_tactic_name(kind: int, tactic: int) -> str:
     return load().bsg_tactic_name(int(kind), int(tactic)).decode()
 
 
-def bsg_choose_tactic(kind, m_rows, segments, N, K, sm_count) -> int:
-    r = int(load().bsg_choose_tactic(int(kind), int(m_rows), int(segments), int(N), int(K), int(sm_count)))
+def bsg_choose_tactic(kind, M, N, K, G, sm_count) -> int:
+    r = int(load().bsg_choose_tactic(int(kind), int(M), int(N), int(K), int(G), int(sm_count)))
     _check(min(r, 0))
     return r
 
 
-def bsg_tactic_score(kind, tactic, m_rows, segments, N, K, sm_count) -> float:
-    return float(load().bsg_tactic_score(int(kind), int(tactic), int(m_rows), int(segments), int(N), int(K),
-                                         int(sm_count)))
+def bsg_tactic_score(kind, tactic, M, N, K, G, sm_count) -> float:
+    return float(load().bsg_tactic_score(int(kind), int(tactic), int(M), int(N), int(K), int(G), int(sm_count)))
 
 
 def bsg_set_tactic(kind: int, tactic: int):

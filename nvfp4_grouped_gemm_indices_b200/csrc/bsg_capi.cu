@@ -51,6 +51,7 @@ struct DeviceState {
   bsg::DeviceStatus* status = nullptr;
   bool fp8_attr = false;
   bool nvfp4_attr = false;
+  int fp8_pair_clusters = 0;
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -157,6 +158,18 @@ bsg_status check_common(const void* A, const void* B, const int32_t* m_indices, 
   return BSG_OK;
 }
 
+// Raster groups of N tiles: when one expert's B (N x K bytes) fits comfortably in L2 the units run
+// window-major (all N tiles of a window together); otherwise N tiles are grouped so that the group's
+// slice of B (about 24 MB) stays resident while every window streams past it.
+int n_group_for(int64_t N, int64_t row_bytes, int bn) {
+  const int64_t n_tiles = (N + bn - 1) / bn;
+  const int64_t b_bytes = N * row_bytes;
+  if (b_bytes <= (48ll << 20)) return static_cast<int>(n_tiles);
+  int64_t g = (24ll << 20) / (static_cast<int64_t>(bn) * row_bytes);
+  if (g < 1) g = 1;
+  return static_cast<int>(g < n_tiles ? g : n_tiles);
+}
+
 int grid_for(int sm_count, int64_t M, int64_t N, int64_t G, int bn) {
   const int64_t n_tiles = (N + bn - 1) / bn;
   const int64_t windows = (M + 127) / 128;
@@ -166,6 +179,7 @@ int grid_for(int sm_count, int64_t M, int64_t N, int64_t G, int bn) {
 }
 
 }  // namespace
+
 
 extern "C" {
 
@@ -213,6 +227,10 @@ bsg_status bsg_fp8_grouped_gemm(const void* A, const void* B, const float* a_sca
   DeviceState* dev = nullptr;
   if ((st = device_state(&dev)) != BSG_OK) return st;
 
+  // tactic 0: one SM per 128 x 256 tile; tactic 1: an SM pair per 256 x 256 tile (cta_group::2)
+  const int tactic = bsg_choose_tactic(0, M, N, K, G, dev->sm_count);
+  const int cg = tactic == 1 ? 2 : 1;
+
   bsg::Fp8Params p;
   memset(&p, 0, sizeof(p));
   {
@@ -225,7 +243,8 @@ bsg_status bsg_fp8_grouped_gemm(const void* A, const void* B, const float* a_sca
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), static_cast<uint64_t>(G)};
     const uint64_t str[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N) * static_cast<uint64_t>(K)};
-    const uint32_t box[3] = {128u, static_cast<uint32_t>(bsg::fp8::BN), 1u};
+    // B rows per CTA and stage: 256 (one SM, 256-column tile) or 64 (each CTA of an SM pair, 128-column tile)
+    const uint32_t box[3] = {128u, static_cast<uint32_t>(cg == 2 ? bsg::fp8::Cfg<2>::B_BOX_ROWS : bsg::fp8::Cfg<1>::B_BOX_ROWS), 1u};
     const bool oob[3] = {false, true, false};  // an N tail tile is zero-filled, columns masked
     if ((st = encode(&p.tmB, "B", B, 3, dims, str, box, oob, CU_TENSOR_MAP_SWIZZLE_128B)) != BSG_OK) return st;
   }
@@ -237,19 +256,64 @@ bsg_status bsg_fp8_grouped_gemm(const void* A, const void* B, const float* a_sca
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.G = static_cast<int>(G);
+  const int bn = cg == 2 ? bsg::fp8::Cfg<2>::BN : bsg::fp8::Cfg<1>::BN;
+  p.n_group = n_group_for(N, K, bn);
   p.timeout_ns = current_timeout();
   p.status = dev->status;
   p.debug_mode = current_fault();
 
   cudaError_t e;
   if (!dev->fp8_attr) {
-    e = cudaFuncSetAttribute(bsg::fp8::kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(bsg::fp8::SMEM_BYTES));
+    e = cudaFuncSetAttribute(bsg::fp8::bsg_fp8_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bsg::fp8::smem_bytes<1>()));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fp8 kernel smem)");
+    e = cudaFuncSetAttribute(bsg::fp8::bsg_fp8_grouped_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bsg::fp8::smem_bytes<2>()));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fp8 2-SM kernel smem)");
+    // how many SM-pair clusters can be resident at once
+    cudaLaunchConfig_t qc = {};
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = 2;
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    qc.gridDim = dim3(2 * (dev->sm_count / 2), 1, 1);
+    qc.blockDim = dim3(bsg::fp8::THREADS, 1, 1);
+    qc.dynamicSmemBytes = bsg::fp8::smem_bytes<2>();
+    qc.attrs = qa;
+    qc.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, bsg::fp8::bsg_fp8_grouped_2sm_kernel, &qc);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(fp8 2-SM kernel)");
+    dev->fp8_pair_clusters = clusters;
     dev->fp8_attr = true;
   }
-  const int grid = bsg_forced_grid(0, grid_for(dev->sm_count, M, N, G, bsg::fp8::BN));
-  bsg::fp8::kernel<<<grid, bsg::fp8::THREADS, bsg::fp8::SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (cg == 1) {
+    const int grid = bsg_forced_grid(0, grid_for(dev->sm_count, M, N, G, bn));
+    bsg::fp8::bsg_fp8_grouped_kernel<<<grid, bsg::fp8::THREADS, bsg::fp8::smem_bytes<1>(), cs>>>(p);
+  } else {
+    if (dev->fp8_pair_clusters < 1) return fail(BSG_ERR_CUDA, "no SM-pair cluster fits on this device");
+    const BsgUnitEstimate est = bsg_estimate_units(M, G);
+    const int64_t n_tiles = (N + bn - 1) / bn;
+    int64_t clusters = est.pairs * n_tiles;
+    if (clusters > dev->fp8_pair_clusters) clusters = dev->fp8_pair_clusters;
+    const int grid = 2 * ((bsg_forced_grid(0, static_cast<int>(2 * clusters)) + 1) / 2);
+    cudaLaunchConfig_t lc = {};
+    cudaLaunchAttribute la[1];
+    la[0].id = cudaLaunchAttributeClusterDimension;
+    la[0].val.clusterDim.x = 2;
+    la[0].val.clusterDim.y = 1;
+    la[0].val.clusterDim.z = 1;
+    lc.gridDim = dim3(grid, 1, 1);
+    lc.blockDim = dim3(bsg::fp8::THREADS, 1, 1);
+    lc.dynamicSmemBytes = bsg::fp8::smem_bytes<2>();
+    lc.stream = cs;
+    lc.attrs = la;
+    lc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&lc, bsg::fp8::bsg_fp8_grouped_2sm_kernel, p);
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the fp8 2-SM grouped kernel");
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launch of the fp8 grouped kernel");
   return BSG_OK;
@@ -309,19 +373,20 @@ bsg_status bsg_nvfp4_gemm(const void* A, const void* B, const void* sfa, const v
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.G = static_cast<int>(G);
+  p.n_group = n_group_for(N, K / 2 + K / 16, bsg::nvfp4::BN);
   p.timeout_ns = current_timeout();
   p.status = dev->status;
   p.debug_mode = current_fault();
 
   cudaError_t e;
   if (!dev->nvfp4_attr) {
-    e = cudaFuncSetAttribute(bsg::nvfp4::kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(bsg::nvfp4::bsg_nvfp4_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(bsg::nvfp4::SMEM_BYTES));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(nvfp4 kernel smem)");
     dev->nvfp4_attr = true;
   }
   const int grid = bsg_forced_grid(1, grid_for(dev->sm_count, M, N, G, bsg::nvfp4::BN));
-  bsg::nvfp4::kernel<<<grid, bsg::nvfp4::THREADS, bsg::nvfp4::SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(
+  bsg::nvfp4::bsg_nvfp4_grouped_kernel<<<grid, bsg::nvfp4::THREADS, bsg::nvfp4::SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(
       p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launch of the nvfp4 kernel");

@@ -3,16 +3,19 @@
 // Score of a tactic (the ranking of the page "[flashinfer] FlashInfer의 FP4 GEMM 최적화: 휴리스틱
 // 개선과 Autotuning 효율화", section 2):
 //     score = m_eff * n_eff * throughput / (num_waves * tile_n)
-//     score *= 1.05            if the tactic issues 2-CTA (cta_group::2) MMAs
-//     score *= 0.95^(log2 cga_n)   for a cluster of cga_n CTAs along N (multicast)
+//     score *= 1.05                 if the tactic issues 2-CTA (cta_group::2) MMAs
+//     score *= 0.95^(log2 cga_n)    for a cluster of cga_n CTAs along N (multicast)
 // The page names but does not define m_eff, n_eff, throughput and num_waves.  Readings used here:
-//     m_eff      = useful rows / rows computed = M_routed / (segments * tile_m)   (window segments are
-//                  the row tiles of this library, so the padding they waste is what m_eff measures)
+//     m_eff      = rows / rows computed: M / (segments * 128) for one-SM tiles, M / (pairs * 256)
+//                  for SM-pair tiles (window segments are the row tiles of this library, so the
+//                  padding they waste is what m_eff measures); segments and pairs are estimated from
+//                  M and G (sorted routing), since m_indices stays on the device
 //     n_eff      = N / (ceil(N / tile_n) * tile_n)
-//     num_waves  = ceil(units / (sm_count / cluster_size)), units = segments * ceil(N / tile_n)
-//     throughput = the tile's relative tensor-core rate (1.0 for the full 128 x 256 issue shape,
-//                  proportionally less for narrower N tiles that leave the pipe shared-memory bound)
-// The exhaustive sweep over all tactics (bench.py --sweep) is what validates the ranking.
+//     num_waves  = ceil(units / (sm_count / cluster_size))
+//     throughput = the tile's sustained fraction of the FP8 / FP4 tensor peak measured on the
+//                  prefill workloads (one-SM FP8 tile 0.44, SM-pair FP8 tile 0.26, NVFP4 0.40);
+//                  the exhaustive sweep re-measures it
+// The sweep over all tactics is what validates the ranking.
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -34,10 +37,11 @@ struct Tactic {
 
 // FP8 and NVFP4 tactic tables (kind 0 and 1).  Only tactics that exist as kernels are listed.
 const Tactic kFp8[] = {
-    {"fp8_1sm_m128_n256_s4", 128, 256, 1, 1, 1.0},
+    {"fp8_1sm_m128_n256_s4", 128, 256, 1, 1, 0.44},
+    {"fp8_2sm_m256_n128_s8", 256, 128, 2, 1, 0.26},
 };
 const Tactic kNvfp4[] = {
-    {"nvfp4_1sm_m128_n256_s4", 128, 256, 1, 1, 1.0},
+    {"nvfp4_1sm_m128_n256_s4", 128, 256, 1, 1, 0.40},
 };
 
 const Tactic* table(int kind, int* n) {
@@ -69,6 +73,15 @@ void read_env() {
 
 }  // namespace
 
+BsgUnitEstimate bsg_estimate_units(int64_t M, int64_t G) {
+  BsgUnitEstimate e;
+  e.windows = (M + 127) / 128;
+  const int64_t runs = G < M ? G : M;
+  e.segments = e.windows + runs - 1;
+  e.pairs = (e.segments + 1) / 2 + runs / 2;
+  return e;
+}
+
 int bsg_forced_grid(int kind, int grid) {
   std::lock_guard<std::mutex> lock(g_mu);
   if (kind < 0 || kind > 1) return grid;
@@ -92,17 +105,19 @@ const char* bsg_tactic_name(int kind, int tactic) {
   return t[tactic].name;
 }
 
-double bsg_tactic_score(int kind, int tactic, int64_t m_rows, int64_t segments, int64_t N, int64_t K, int sm_count) {
+double bsg_tactic_score(int kind, int tactic, int64_t M, int64_t N, int64_t K, int64_t G, int sm_count) {
   (void)K;
   int n = 0;
   const Tactic* tt = table(kind, &n);
-  if (!tt || tactic < 0 || tactic >= n || m_rows <= 0 || segments <= 0 || N <= 0 || sm_count <= 0) return 0.0;
+  if (!tt || tactic < 0 || tactic >= n || M <= 0 || N <= 0 || G <= 0 || sm_count <= 0) return 0.0;
   const Tactic& t = tt[tactic];
+  const BsgUnitEstimate est = bsg_estimate_units(M, G);
+  const double row_tiles = static_cast<double>(t.cta_group == 2 ? est.pairs : est.segments);
   const double tiles_n = std::ceil(static_cast<double>(N) / t.tile_n);
-  const double m_eff = static_cast<double>(m_rows) / (static_cast<double>(segments) * t.tile_m);
+  const double m_eff = static_cast<double>(M) / (row_tiles * t.tile_m);
   const double n_eff = static_cast<double>(N) / (tiles_n * t.tile_n);
   const int cluster = t.cta_group * t.cga_n;
-  const double units = static_cast<double>(segments) * tiles_n / t.cta_group;
+  const double units = row_tiles * tiles_n;
   const double slots = std::floor(static_cast<double>(sm_count) / cluster);
   const double waves = std::ceil(units / (slots > 0 ? slots : 1.0));
   double score = m_eff * n_eff * t.throughput / (waves * t.tile_n);
@@ -113,7 +128,7 @@ double bsg_tactic_score(int kind, int tactic, int64_t m_rows, int64_t segments, 
   return score;
 }
 
-int bsg_choose_tactic(int kind, int64_t m_rows, int64_t segments, int64_t N, int64_t K, int sm_count) {
+int bsg_choose_tactic(int kind, int64_t M, int64_t N, int64_t K, int64_t G, int sm_count) {
   int n = 0;
   if (!table(kind, &n)) return BSG_ERR_INVALID_ARG;
   {
@@ -125,9 +140,9 @@ int bsg_choose_tactic(int kind, int64_t m_rows, int64_t segments, int64_t N, int
   int best = 0;
   double best_score = -1.0;
   for (int i = 0; i < n; ++i) {
-    double s = bsg_tactic_score(kind, i, m_rows, segments, N, K, sm_count);
-    if (s > best_score) {
-      best_score = s;
+    double sc = bsg_tactic_score(kind, i, M, N, K, G, sm_count);
+    if (sc > best_score) {
+      best_score = sc;
       best = i;
     }
   }

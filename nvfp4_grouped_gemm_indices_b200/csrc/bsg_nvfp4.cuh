@@ -40,6 +40,7 @@ struct Nvfp4Params {
   const int* m_indices;
   __nv_bfloat16* C;
   int M, N, K, G;
+  int n_group;        // N tiles per raster group
   uint64_t timeout_ns;
   DeviceStatus* status;
   int debug_mode;
@@ -109,7 +110,7 @@ __device__ __forceinline__ void shuffle_sf_block(uint8_t* blk) {
   *reinterpret_cast<uint4*>(blk + 3 * 512 + l * 16) = o3;
 }
 
-__global__ void __launch_bounds__(THREADS, 1) kernel(const __grid_constant__ Nvfp4Params p) {
+__global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __grid_constant__ Nvfp4Params p) {
   extern __shared__ uint8_t smem_raw[];
   Smem& s = smem_ref(smem_raw);
   const int warp = warp_idx();
@@ -153,7 +154,7 @@ __global__ void __launch_bounds__(THREADS, 1) kernel(const __grid_constant__ Nvf
   const uint32_t tmem_base = s.tmem_base;
 
   if (warp == WARP_SCHED) {
-    run_scheduler<Q, BN>(s.queue, p.m_indices, p.M, p.G, n_tiles, wctx, p.debug_mode);
+    run_scheduler<Q, BN, false>(s.queue, p.m_indices, p.M, p.G, n_tiles, p.n_group, wctx, p.debug_mode);
   } else if (warp == WARP_TMA) {
     int qslot = 0;
     uint32_t qphase = 0;

@@ -116,71 +116,144 @@ __device__ __forceinline__ int routed_expert(const int* __restrict__ m_indices, 
   return (g >= 0 && g < G) ? g : -1;
 }
 
-// Scheduler warp body.  n_tiles = ceil(N / BN).
-template <int Q, int BN>
+// Scheduler warp body.  n_tiles = ceil(N / BN); n_group = N tiles per raster group.
+//
+// Unit order: for each group of n_group consecutive N tiles, for each window, for each segment of
+// the window, for each N tile of the group.  With n_group = n_tiles this is window-major (the rows
+// of a window are reused from L2 across all N tiles, and B[g] across the windows of an expert);
+// smaller groups keep a slice of a large B resident while all windows stream past it.
+// The m_indices of kScanBatch windows are loaded at once, so walking to a CTA's first unit costs
+// one memory latency per kScanBatch windows.
+//
+// PAIR = false: one CTA per unit; CTA b of P takes units b, b + P, ...
+// PAIR = true : two CTAs (a cluster pair) per unit.  Consecutive segments (in window order) of the
+// same expert are paired -- a run spanning several windows gives pairs of consecutive windows -- and
+// a segment without a partner is paired with an empty half (rows [0, 0): computed, never stored).
+// Cluster c of P/2 takes pair-units c, c + P/2, ...; CTA rank r of the pair receives half r.
+constexpr int kScanBatch = 4;
+
+struct Seg {
+  int row0, lo, hi, g;
+};
+
+template <int Q, int BN, bool PAIR>
 __device__ void run_scheduler(UnitQueue<Q>& q, const int* __restrict__ m_indices, int M, int G, int n_tiles,
-                              const WaitCtx& wctx, int debug_mode) {
+                              int n_group, const WaitCtx& wctx, int debug_mode) {
   if (debug_mode == kDebugWithholdSchedule) return;
   const int lane = lane_idx();
   const unsigned FULL = 0xffffffffu;
   int slot = 0;
   uint32_t phase = 0;
-  long long next = blockIdx.x;           // next global unit index this CTA owns
-  const long long stride = gridDim.x;
-  long long first = 0;                   // global index of the first unit of the current window
+  const long long owner = PAIR ? blockIdx.x / 2 : blockIdx.x;   // cluster (pair) or CTA index
+  const long long stride = PAIR ? gridDim.x / 2 : gridDim.x;
+  const int half = PAIR ? static_cast<int>(blockIdx.x & 1) : 0;
+  long long next = owner;                 // next global unit index this CTA (pair) owns
+  long long first = 0;                    // global index of the first unit of the next segment/pair
   const int n_windows = (M + 127) / 128;
-  for (int w = 0; w < n_windows; ++w) {
-    const int row0 = w * 128;
-    int gj[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) gj[j] = routed_expert(m_indices, row0 + 32 * j + lane, M, G);
-    uint32_t smask[4], emask[4];
-    int nseg = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      int prev = __shfl_up_sync(FULL, gj[j], 1);
-      int nxt = __shfl_down_sync(FULL, gj[j], 1);
-      int prev_chunk_last = (j > 0) ? __shfl_sync(FULL, gj[j > 0 ? j - 1 : 0], 31) : -1;
-      int next_chunk_first = (j < 3) ? __shfl_sync(FULL, gj[j < 3 ? j + 1 : 3], 0) : -1;
-      if (lane == 0) prev = prev_chunk_last;
-      if (lane == 31) nxt = next_chunk_first;
-      const bool is_start = gj[j] >= 0 && gj[j] != prev;
-      const bool is_end = gj[j] >= 0 && gj[j] != nxt;
-      smask[j] = __ballot_sync(FULL, is_start);
-      emask[j] = __ballot_sync(FULL, is_end);
-      nseg += __popc(smask[j]);
+  const int n_groups = (n_tiles + n_group - 1) / n_group;
+  bool alive = true;
+
+  // hand out the units [first, first + tiles) that this CTA owns; returns false on abort
+  auto emit = [&](const Seg& a, const Seg* b, int t0, int tiles) -> bool {
+    const long long base = first;
+    first += tiles;
+    if (next >= base + tiles) return true;
+    Unit u;
+    const Seg* mine = (half == 0) ? &a : b;
+    if (mine) {
+      u.row0 = mine->row0;
+      u.row_lo = mine->lo;
+      u.row_hi = mine->hi;
+    } else {
+      u.row0 = a.row0;  // empty half: load the partner's window, store nothing
+      u.row_lo = 0;
+      u.row_hi = 0;
     }
-    const long long units_here = static_cast<long long>(nseg) * n_tiles;
-    if (next >= first + units_here) {
-      first += units_here;
-      continue;
+    u.g = a.g;
+    u.valid = 1;
+    u.pad0 = u.pad1 = 0;
+    while (next < base + tiles) {
+      u.n0 = (t0 + static_cast<int>(next - base)) * BN;
+      if (!queue_push(q, slot, phase, u, wctx)) return false;
+      next += stride;
     }
-    int js = 0, je = 0;
-    uint32_t ms = smask[0], me = emask[0];
-    for (int k = 0; k < nseg; ++k) {
-      while (ms == 0) { ++js; ms = smask[js]; }
-      while (me == 0) { ++je; me = emask[je]; }
-      const int bs = __ffs(ms) - 1;
-      const int be = __ffs(me) - 1;
-      ms &= ms - 1;
-      me &= me - 1;
-      const long long base = first + static_cast<long long>(k) * n_tiles;
-      if (next >= base + n_tiles) continue;
-      Unit u;
-      u.row0 = row0;
-      u.row_lo = row0 + 32 * js + bs;
-      u.row_hi = row0 + 32 * je + be + 1;
-      u.g = m_indices ? __ldg(m_indices + u.row_lo) : 0;
-      u.valid = 1;
-      u.pad0 = u.pad1 = 0;
-      while (next < base + n_tiles) {
-        u.n0 = static_cast<int>(next - base) * BN;
-        if (!queue_push(q, slot, phase, u, wctx)) return;
-        next += stride;
+    return true;
+  };
+
+  for (int grp = 0; grp < n_groups && alive; ++grp) {
+    const int t0 = grp * n_group;
+    const int tiles = min(n_group, n_tiles - t0);
+    Seg pending;
+    bool have_pending = false;
+    for (int wb = 0; wb < n_windows && alive; wb += kScanBatch) {
+      int gv[kScanBatch][4];
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) gv[i][j] = routed_expert(m_indices, (wb + i) * 128 + 32 * j + lane, M, G);
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i) {
+        const int w = wb + i;
+        if (w >= n_windows || !alive) break;
+        const int row0 = w * 128;
+        uint32_t smask[4], emask[4];
+        int nseg = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          int prev = __shfl_up_sync(FULL, gv[i][j], 1);
+          int nxt = __shfl_down_sync(FULL, gv[i][j], 1);
+          const int prev_chunk_last = __shfl_sync(FULL, gv[i][j > 0 ? j - 1 : 0], 31);
+          const int next_chunk_first = __shfl_sync(FULL, gv[i][j < 3 ? j + 1 : 3], 0);
+          if (lane == 0) prev = (j > 0) ? prev_chunk_last : -1;
+          if (lane == 31) nxt = (j < 3) ? next_chunk_first : -1;
+          const bool is_start = gv[i][j] >= 0 && gv[i][j] != prev;
+          const bool is_end = gv[i][j] >= 0 && gv[i][j] != nxt;
+          smask[j] = __ballot_sync(FULL, is_start);
+          emask[j] = __ballot_sync(FULL, is_end);
+          nseg += __popc(smask[j]);
+        }
+        if (!PAIR) {
+          // every segment is a unit: skip the window in one step when this CTA owns none of it
+          const long long units_here = static_cast<long long>(nseg) * tiles;
+          if (next >= first + units_here) {
+            first += units_here;
+            continue;
+          }
+        }
+        int js = 0, je = 0;
+        uint32_t ms = smask[0], me = emask[0];
+        for (int k = 0; k < nseg; ++k) {
+          while (ms == 0) { ++js; ms = smask[js]; }
+          while (me == 0) { ++je; me = emask[je]; }
+          const int bs = __ffs(ms) - 1;
+          const int be = __ffs(me) - 1;
+          ms &= ms - 1;
+          me &= me - 1;
+          const int gsel = js == 0 ? gv[i][0] : js == 1 ? gv[i][1] : js == 2 ? gv[i][2] : gv[i][3];
+          Seg sg;
+          sg.row0 = row0;
+          sg.lo = row0 + 32 * js + bs;
+          sg.hi = row0 + 32 * je + be + 1;
+          sg.g = __shfl_sync(FULL, gsel, bs);
+          if (!PAIR) {
+            if (!emit(sg, nullptr, t0, tiles)) alive = false;
+          } else if (have_pending && pending.g == sg.g) {
+            if (!emit(pending, &sg, t0, tiles)) alive = false;
+            have_pending = false;
+          } else {
+            if (have_pending && !emit(pending, nullptr, t0, tiles)) alive = false;
+            pending = sg;
+            have_pending = true;
+          }
+          if (!alive) break;
+        }
       }
     }
-    first += units_here;
+    if (PAIR && have_pending && alive) {
+      if (!emit(pending, nullptr, t0, tiles)) alive = false;
+    }
   }
+  if (!alive) return;
   Unit done;
   done.row0 = done.row_lo = done.row_hi = done.g = done.n0 = 0;
   done.valid = 0;

@@ -120,21 +120,44 @@ def test_timeout_setter_roundtrip(lib):
 
 
 def test_chooser_score_follows_the_page_formula(lib):
+    """score = m_eff * n_eff * throughput / (num_waves * tile_n), x1.05 for 2-SM tactics."""
     for kind in (0, 1):
         n = bsg.bsg_num_tactics(kind)
         assert n >= 1
         for t in range(n):
             assert bsg.bsg_tactic_name(kind, t)
-            s = bsg.bsg_tactic_score(kind, t, 8192, 71, 4096, 7168, 148)
-            assert s > 0
-        best = bsg.bsg_choose_tactic(kind, 8192, 71, 4096, 7168, 148)
-        scores = [bsg.bsg_tactic_score(kind, t, 8192, 71, 4096, 7168, 148) for t in range(n)]
+            assert bsg.bsg_tactic_score(kind, t, 8192, 4096, 7168, 8, 148) > 0
+        best = bsg.bsg_choose_tactic(kind, 8192, 4096, 7168, 8, 148)
+        scores = [bsg.bsg_tactic_score(kind, t, 8192, 4096, 7168, 8, 148) for t in range(n)]
         assert best == max(range(n), key=lambda t: scores[t])
-    # a single-tactic check of the formula: 64 full windows, N = 4096, tile 128 x 256, 148 SMs
-    s = bsg.bsg_tactic_score(0, 0, 8192, 64, 4096, 7168, 148)
-    waves = -(-(64 * 16) // 148)
-    assert abs(s - 1.0 * 1.0 * 1.0 / (waves * 256)) < 1e-15
-    assert bsg.bsg_tactic_score(0, 99, 1, 1, 64, 128, 148) == 0.0
+    # FP8 one-SM tactic 0 on M=8192 (64 windows), G=8: 71 segments, N=4096 -> 16 tiles of 256
+    thr = {"fp8_1sm_m128_n256_s4": 0.44, "fp8_2sm_m256_n128_s8": 0.26}
+    assert bsg.bsg_tactic_name(0, 0) in thr
+    segs, pairs = 64 + 8 - 1, (64 + 8 - 1 + 1) // 2 + 8 // 2
+    t0 = bsg.bsg_tactic_name(0, 0)
+    s = bsg.bsg_tactic_score(0, 0, 8192, 4096, 7168, 8, 148)
+    waves = -(-(segs * 16) // 148)
+    assert abs(s - (8192 / (segs * 128)) * thr[t0] / (waves * 256)) < 1e-15
+    if bsg.bsg_num_tactics(0) > 1:
+        t1 = bsg.bsg_tactic_name(0, 1)
+        s1 = bsg.bsg_tactic_score(0, 1, 8192, 4096, 7168, 8, 148)
+        waves1 = -(-(pairs * 32) // 74)
+        assert abs(s1 - (8192 / (pairs * 256)) * thr[t1] * 1.05 / (waves1 * 128)) < 1e-15
+        # a skewed, tiny-M routing over many experts leaves 2-SM tiles half empty: one SM wins
+        assert bsg.bsg_choose_tactic(0, 512, 4096, 7168, 64, 148) == 0
+        # with the measured tile throughputs the one-SM tile wins the prefill shape as well
+        assert bsg.bsg_choose_tactic(0, 8192, 4096, 7168, 8, 148) == 0
+    assert bsg.bsg_tactic_score(0, 99, 1, 64, 128, 1, 148) == 0.0
+
+
+def test_tactic_override(lib):
+    try:
+        bsg.bsg_set_tactic(0, 0)
+        assert bsg.bsg_choose_tactic(0, 8192, 4096, 7168, 8, 148) == 0
+    finally:
+        bsg.bsg_set_tactic(0, -1)
+    with pytest.raises(bsg.BsgError):
+        bsg.bsg_set_tactic(0, 99)
 
 
 def test_set_max_ctas_validation(lib):

@@ -15,6 +15,17 @@ from gpu_util import (SENTINEL, DevWorkload, bits, compare, oracle_rows, routed_
 
 pytestmark = pytest.mark.gpu
 
+FP8_TACTICS = [0, 1]  # 0: one SM per 128 x 256 tile; 1: an SM pair per 256 x 256 tile (cta_group::2)
+
+
+@pytest.fixture(params=FP8_TACTICS, ids=lambda t: f"tactic{t}")
+def tactic(request):
+    if request.param >= bsg.bsg_num_tactics(0):
+        pytest.skip("tactic not built")
+    bsg.bsg_set_tactic(0, request.param)
+    yield request.param
+    bsg.bsg_set_tactic(0, -1)
+
 
 def full_check(w):
     d = DevWorkload(w)
@@ -25,13 +36,13 @@ def full_check(w):
     return compare(out, ref, routed_mask(w))
 
 
-def test_fp8_small_workload_full():
+def test_fp8_small_workload_full(tactic):
     """4 experts, M=512, N=256, K=512; run boundaries inside 128-row windows."""
     full_check(W.config(0))
 
 
 @pytest.mark.parametrize("M,N,K,G,ctas", [(65, 128, 128, 2, 4), (777, 256, 512, 8, 84)])
-def test_fp8_page_benchmark_shapes(M, N, K, G, ctas):
+def test_fp8_page_benchmark_shapes(M, N, K, G, ctas, tactic):
     """The two shapes of the FP8 page's benchmark table, balanced sorted runs."""
     counts = [M // G + (1 if i < M % G else 0) for i in range(G)]
     w = W.make_fp8(M, N, K, G, W.counts_to_indices(counts), seed=M)
@@ -63,7 +74,7 @@ def _routing(case, M, G, rng):
 
 
 @pytest.mark.parametrize("case", ["sorted", "len1_runs", "empty_experts", "span3windows", "skip_rows", "unsorted"])
-def test_fp8_routing_edge_cases(case):
+def test_fp8_routing_edge_cases(case, tactic):
     rng = np.random.default_rng(hash(case) % 1000)
     M, N, K, G = 400, 256, 256, 5
     w = W.make_fp8(M, N, K, G, _routing(case, M, G, rng), seed=7)
@@ -71,7 +82,7 @@ def test_fp8_routing_edge_cases(case):
 
 
 @pytest.mark.parametrize("M", [1, 127, 128, 129, 300])
-def test_fp8_row_counts(M):
+def test_fp8_row_counts(M, tactic):
     G = 3 if M > 2 else 1
     rng = np.random.default_rng(M)
     idx = W.counts_to_indices(rng.multinomial(M, [1.0 / G] * G)) if G > 1 else np.zeros(M, np.int32)
@@ -79,20 +90,20 @@ def test_fp8_row_counts(M):
     full_check(w)
 
 
-def test_fp8_single_expert_null_indices():
+def test_fp8_single_expert_null_indices(tactic):
     w = W.make_fp8(200, 256, 256, 1, None, seed=3)
     full_check(w)
 
 
 @pytest.mark.parametrize("N", [64, 136, 264, 520])
-def test_fp8_n_tails(N):
+def test_fp8_n_tails(N, tactic):
     rng = np.random.default_rng(N)
     idx = W.counts_to_indices(rng.multinomial(300, [0.5, 0.5]))
     w = W.make_fp8(300, N, 256, 2, idx, seed=N)
     full_check(w)
 
 
-def test_fp8_many_experts_mostly_empty():
+def test_fp8_many_experts_mostly_empty(tactic):
     """G = 64 with a Zipf routing of 512 rows: many experts with 0-3 rows."""
     rng = np.random.default_rng(11)
     idx = W.routing_zipf(512, 64, rng)
@@ -100,7 +111,7 @@ def test_fp8_many_experts_mostly_empty():
     full_check(w)
 
 
-def test_fp8_integer_grid_bit_exact():
+def test_fp8_integer_grid_bit_exact(tactic):
     """Small integer codes and power-of-two scales: every sum is exact in fp32, so the GPU result
     must equal the oracle's bf16 bit for bit."""
     rng = np.random.default_rng(5)
@@ -122,7 +133,7 @@ def test_fp8_integer_grid_bit_exact():
 
 
 @pytest.mark.parametrize("ctas", [1, 2, 3, 7])
-def test_fp8_persistent_grid_sizes_bit_identical(ctas):
+def test_fp8_persistent_grid_sizes_bit_identical(ctas, tactic):
     """Each CTA walks many units through the same rings (stage counts that do not divide the
     number of K blocks): the result must not depend on the grid size."""
     rng = np.random.default_rng(21)
@@ -139,7 +150,7 @@ def test_fp8_persistent_grid_sizes_bit_identical(ctas):
     compare(ref, oracle_rows(w), routed_mask(w))
 
 
-def test_fp8_graph_replay_sees_new_indices():
+def test_fp8_graph_replay_sees_new_indices(tactic):
     """m_indices is read on the device at every launch: a captured graph replayed after the routing
     (and the data) changed in place computes the new result."""
     rng = np.random.default_rng(8)
@@ -168,7 +179,7 @@ def test_fp8_graph_replay_sees_new_indices():
 
 
 @pytest.mark.parametrize("cfg", [1, 4])
-def test_fp8_full_size_sampled_rows(cfg):
+def test_fp8_full_size_sampled_rows(cfg, tactic):
     """The full-size FP8 workloads (MoE prefill G=8 M=8192 N=4096 K=7168; decode-like Zipf G=64
     M=512 N=4096 K=7168) in the benchmark's launch configuration, checked on every row near a run
     boundary plus random rows (all N columns); every other row is checked for NaN/sentinel."""
