@@ -16,11 +16,9 @@
 //           ahead of the promotion instead of one, which hides the commit -> promote -> release
 //           hand-off latency (measured ~700 cycles against a 512-cycle MMA block).
 // Roles:
-//   warp 0      producer: TMA of the A box [128 rows x 128 B] and this CTA's B box [256/CG rows x
+//   warp 0      producer: TMA of the A box [128 rows x 128 B] and this CTA's B box [BN/CG rows x
 //               128 B] into a STAGES-deep shared-memory ring; the arrival bytes of both CTAs of a
-//               pair count on the even CTA's full barrier.  It also cp.async-s the K block's scales
-//               (a_scale of the 128 rows, b_scale of the tile's two 128-column blocks) into a
-//               separate, deeper scale ring (cp.async.mbarrier.arrive).
+//               pair count on the even CTA's full barrier.
 //   warp 1      TMEM allocator + (even CTA) single-thread tcgen05.mma issuer: per 128-K block, 4 K steps
 //               of kind::f8f6f4 MMAs into a fresh FP32 accumulator: one 128 x 256 MMA per step (CG 1,
 //               two accumulators of 256 columns that ping-pong), or two 256 x 128 MMAs per step, one
@@ -28,7 +26,10 @@
 //               cores run ahead of the epilogue that promotes the previous block.  Completion is
 //               committed to the barriers of both CTAs.
 //   warp 2      scheduler (bsg_sched.cuh): window segmentation, pairing, unit hand-out.
-//   warp 3      idles (20 warps allocate registers like 19: five warps sit on one sub-partition).
+//   warp 3      scale producer: cp.async of each K block's scales (a_scale of the 128 rows, b_scale
+//               of the tile's 128-column blocks) into a separate, deeper scale ring that completes
+//               on an mbarrier (cp.async.mbarrier.arrive).  Kept off the TMA producer's
+//               sub-partition: there its scattered loads delayed the co-resident epilogue warps.
 //   warps 4..19 epilogue (16 warps, 4 per SM sub-partition): warp w owns TMEM lanes 32*(w%4)..
 //               (tile rows) and 64 columns; per K block it reads the fresh partial from TMEM and
 //               accumulates partial * a_scale[row, kb] * b_scale[g, col/128, kb] into registers with
@@ -67,7 +68,7 @@ constexpr int BM = 128;                 // rows per CTA
 constexpr int BK = 128;                 // one scale block
 constexpr int SC_STAGES = 12;           // scale ring: >= STAGES + ACC + slack
 constexpr int Q = 4;                    // unit queue depth
-constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_SCHED = 2, WARP_EPI0 = 4;
+constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_SCHED = 2, WARP_SCALE = 3, WARP_EPI0 = 4;
 constexpr int EPI_WARPS = 16;
 constexpr int NUM_WARPS = WARP_EPI0 + EPI_WARPS;
 constexpr int THREADS = NUM_WARPS * 32;
@@ -164,7 +165,7 @@ __device__ __forceinline__ void fp8_kernel_body(const Fp8Params& p) {
     }
     for (int i = 0; i < Q; ++i) {
       mbar_init(&s.queue.full[i], 1);
-      mbar_init(&s.queue.empty[i], EPI_WARPS + 2);
+      mbar_init(&s.queue.empty[i], EPI_WARPS + 3);
     }
     mbar_init(&s.mma_done, 1);
     s.abort = 0;
@@ -194,13 +195,15 @@ __device__ __forceinline__ void fp8_kernel_body(const Fp8Params& p) {
 
   if (warp == WARP_SCHED) {
     run_scheduler<Q, BN, CG == 2>(s.queue, p.m_indices, p.M, p.G, n_tiles, p.n_group, wctx, p.debug_mode);
-  } else if (warp == WARP_TMA) {
+  } else if (warp == WARP_SCALE) {
+    // scale producer: the K block's a_scale (128 rows of the window) and b_scale (the tile's
+    // 128-column blocks) by cp.async into the scale ring; a warp of its own keeps these scattered
+    // 4-byte loads off the sub-partition of the TMA producer
     const int NB = (p.N + 127) / 128;
     int qslot = 0;
     uint32_t qphase = 0;
-    RingPos<STAGES> pos;
     RingPos<SC_STAGES> spos;
-    long long issued = 0, sc_issued = 0;
+    long long issued = 0;
     bool ok = true;
     while (ok) {
       Unit u;
@@ -210,6 +213,43 @@ __device__ __forceinline__ void fp8_kernel_body(const Fp8Params& p) {
       }
       if (!u.valid) break;
       const int nb0 = u.n0 / 128;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&s.sc_empty[spos.stage], spos.phase ^ 1u, wctx.timeout_ns, wctx.abort, wctx.status,
+                       kSiteSmemEmpty, 16 + spos.stage)) {
+          ok = false;
+          break;
+        }
+        ScaleSlot& slot = s.sc[spos.stage];
+#pragma unroll
+        for (int i = 0; i < BM / 32; ++i) {
+          const int row = u.row0 + i * 32 + lane;
+          const bool in = row < p.M;
+          cp_async_4(&slot.a[i * 32 + lane], p.a_scale + static_cast<size_t>(in ? row : 0) * KB + kb, in ? 4u : 0u);
+        }
+        if (lane < C::NB_TILE) {
+          const bool in = nb0 + lane < NB;
+          cp_async_4(&slot.b[lane], p.b_scale + (static_cast<size_t>(u.g) * NB + (in ? nb0 + lane : 0)) * KB + kb,
+                     in ? 4u : 0u);
+        }
+        cp_async_arrive(&s.sc_full[spos.stage]);
+        ++issued;
+        spos.advance();
+      }
+    }
+    if (!ok) drain_inflight_loads<SC_STAGES>(s.sc_full, spos, issued, wctx);
+  } else if (warp == WARP_TMA) {
+    int qslot = 0;
+    uint32_t qphase = 0;
+    RingPos<STAGES> pos;
+    long long issued = 0;
+    bool ok = true;
+    while (ok) {
+      Unit u;
+      if (!queue_pop(s.queue, qslot, qphase, u, wctx)) {
+        ok = false;
+        break;
+      }
+      if (!u.valid) break;
       for (int kb = 0; kb < KB; ++kb) {
         if (!mbar_wait(&s.empty[pos.stage], pos.phase ^ 1u, wctx.timeout_ns, wctx.abort, wctx.status,
                        kSiteSmemEmpty, pos.stage)) {
@@ -233,27 +273,6 @@ __device__ __forceinline__ void fp8_kernel_body(const Fp8Params& p) {
         __syncwarp();
         ++issued;
         pos.advance();
-        // scales of this K block: the 128 rows of the window, the tile's column blocks
-        if (!mbar_wait(&s.sc_empty[spos.stage], spos.phase ^ 1u, wctx.timeout_ns, wctx.abort, wctx.status,
-                       kSiteSmemEmpty, 16 + spos.stage)) {
-          ok = false;
-          break;
-        }
-        ScaleSlot& slot = s.sc[spos.stage];
-#pragma unroll
-        for (int i = 0; i < BM / 32; ++i) {
-          const int row = u.row0 + i * 32 + lane;
-          const bool in = row < p.M;
-          cp_async_4(&slot.a[i * 32 + lane], p.a_scale + static_cast<size_t>(in ? row : 0) * KB + kb, in ? 4u : 0u);
-        }
-        if (lane < C::NB_TILE) {
-          const bool in = nb0 + lane < NB;
-          cp_async_4(&slot.b[lane], p.b_scale + (static_cast<size_t>(u.g) * NB + (in ? nb0 + lane : 0)) * KB + kb,
-                     in ? 4u : 0u);
-        }
-        cp_async_arrive(&s.sc_full[spos.stage]);
-        ++sc_issued;
-        spos.advance();
       }
     }
     if (ok) {
@@ -268,7 +287,6 @@ __device__ __forceinline__ void fp8_kernel_body(const Fp8Params& p) {
       // (CG 2: the odd CTA's loads land on the even CTA's barrier; the closing cluster barrier keeps
       // this CTA's shared memory alive until the even CTA has drained those too.)
       if (CG == 1 || rank == 0) drain_inflight_loads<STAGES>(s.full, pos, issued, wctx);
-      drain_inflight_loads<SC_STAGES>(s.sc_full, spos, sc_issued, wctx);
     }
   } else if (warp == WARP_MMA) {
     constexpr uint32_t IDESC = idesc_f8f6f4_e4m3(BM * CG, BN);
