@@ -4,24 +4,30 @@
 // (SM120+)에서 NVFP4 QMoE를 위한 네이티브 FP4xFP4 Prefill 최적화", section 1:
 //   C[m, n] = bf16( alpha[g] * sum_j sfa[m, j] * sfb[g, n, j] * (A[m, block j] . B[g, n, block j]) )
 //
-// Design (persistent, warp-specialised, one CTA per SM; same skeleton as the FP8 kernel):
-//   warps 0..7  epilogue: after the last K stage of a unit, read the 128 x BN FP32 accumulator from
-//               TMEM (warp w: lanes 32*(w%4).., columns 128*(w/4)..), release it, multiply by
-//               alpha[g], round to BF16, store the segment's rows.
-//   warp 8      TMA producer for A and B (K stage = 256 elements = 128 packed bytes, 128B swizzle).
-//   warp 9      TMEM allocator + single-thread issuer: per K stage, tcgen05.cp of the stage's scale
-//               factors into TMEM, then 4 x (128 x BN x 64) kind::mxf4nvf4 block16 MMAs accumulating
-//               the whole K in one TMEM accumulator (hardware block scaling).
-//   warp 10     scheduler (bsg_sched.cuh).
-//   warp 11     scale-factor producer: TMA of the row-major scale bytes of the stage (sfa: 128 rows x
-//               16 B, sfb: BN rows x 16 B) and an in-place shuffle into the layout tcgen05.cp takes
-//               (for each 64-K MMA step, 32 rows of 16 B each holding rows r, r+32, r+64, r+96),
-//               then a fence to the async proxy and an arrival on the stage's sf_full barrier.  A
-//               separate warp for the scale factors follows the warp-role split of the page
-//               "[cutlass] NVIDIA CUTLASS CuTeDSL: SM103 Grouped Block-Scaled GEMM 최적화 분석",
-//               section 1.
-// TMEM columns: [0, BN) accumulator, [256, 272) SFA (4 columns per MMA step), [272, 304) SFB
-// (8 columns per MMA step for BN = 256).
+// Design (persistent, warp-specialised, one CTA per SM):
+//   warps 0..7   epilogue: after the last K stage of a unit, read the 128 x BN FP32 accumulator from
+//                TMEM (warp w: lanes 32*(w%4).., columns 128*(w/4)..), scale by alpha[g] and pack to
+//                BF16 while reading, release the accumulator, then store the segment's rows.
+//   warp 8       TMA producer for A and B (K stage = 256 elements = 128 packed bytes, 128B swizzle);
+//                it also loads the stage's row-major scale bytes (sfa: 128 rows x 16 B, sfb: BN rows
+//                x 16 B) with TMA into a raw per-stage buffer.
+//   warp 9       TMEM allocator + single-thread issuer: per K stage, 4 x (128 x BN x 64)
+//                kind::mxf4nvf4 block16 MMAs accumulating the whole K in one TMEM accumulator, the
+//                scale factors read from the stage's TMEM scale slot (hardware block scaling).
+//   warp 10      scheduler (bsg_sched.cuh).
+//   warps 11..14 scale-factor writers, one per SM sub-partition (warp % 4 = TMEM lane quarter):
+//                read the stage's raw scale bytes from shared memory into registers, rearrange them
+//                and write them with tcgen05.st into the stage's TMEM scale slot, then arrive on the
+//                stage's `full` barrier next to the TMA bytes.  Separate scale-factor warps follow
+//                the warp-role split of the page "[cutlass] NVIDIA CUTLASS CuTeDSL: SM103 Grouped
+//                Block-Scaled GEMM 최적화 분석", section 1.  Writing TMEM from registers keeps the
+//                scale copies off the tensor pipe: a tcgen05.cp occupies the tensor pipe for about a
+//                third of an MMA's time and does not overlap the MMAs (12 per stage cost ~70% of the
+//                stage's MMA time when measured alone).
+// TMEM columns: [0, BN) accumulator; scale slot s (one per pipeline stage) at 256 + 48 s: SFA in
+// 16 columns (4 per 64-K MMA step), SFB in 32 columns (8 per step).  A step's scales are replicated
+// in all four lane quarters: lane 32q + l, column c of SFA holds the 4 scales of row 32c + l; SFB
+// column c holds those of row 32c + l (c < 8).  Each scale warp writes its own quarter.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -32,9 +38,9 @@
 namespace bsg {
 
 struct Nvfp4Params {
-  CUtensorMap tmA;    // uint8 [M, K/2]:   dims {K/2, M},     box {128, 128},  128B swizzle
-  CUtensorMap tmB;    // uint8 [G, N, K/2]: dims {K/2, N, G}, box {128, BN, 1}, 128B swizzle
-  CUtensorMap tmSFA;  // uint8 [M, K/16]:  dims {K/16, M},    box {16, 128}
+  CUtensorMap tmA;  // uint8 [M, K/2]:    dims {K/2, M},    box {128, 128},  128B swizzle
+  CUtensorMap tmB;  // uint8 [G, N, K/2]: dims {K/2, N, G}, box {128, BN, 1}, 128B swizzle
+  CUtensorMap tmSFA;  // uint8 [M, K/16]:    dims {K/16, M},    box {16, 128}
   CUtensorMap tmSFB;  // uint8 [G, N, K/16]: dims {K/16, N, G}, box {16, BN, 1}
   const float* alpha;
   const int* m_indices;
@@ -54,27 +60,27 @@ constexpr int BK = 256;                  // K elements per stage (128 packed byt
 constexpr int STAGES = 4;
 constexpr int Q = 4;
 constexpr int EPI_WARPS = 8;
-constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_SCHED = 10, WARP_SF = 11;
-constexpr int NUM_WARPS = 12;
+constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_SCHED = 10, WARP_SF0 = 11;
+constexpr int SF_WARPS = 4;
+constexpr int NUM_WARPS = WARP_SF0 + SF_WARPS;
 constexpr int THREADS = NUM_WARPS * 32;
 constexpr int A_BYTES = BM * BK / 2;     // 16 KB
 constexpr int B_BYTES = BN * BK / 2;     // 32 KB
 constexpr int SFA_BYTES = BM * BK / 16;  // 2 KB
 constexpr int SFB_BYTES = BN * BK / 16;  // 4 KB
-constexpr int SF_LAG = STAGES - 1;       // scale stages in flight before the first shuffle
 constexpr int TMEM_COLS = 512;
-constexpr uint32_t COL_SFA = 256;
-constexpr uint32_t COL_SFB = 272;
+constexpr uint32_t COL_SF0 = 256;        // first scale slot
+constexpr uint32_t SF_SLOT_COLS = 48;    // 16 SFA + 32 SFB columns per stage
+constexpr uint32_t SFB_OFF = 16;
+static_assert(COL_SF0 + STAGES * SF_SLOT_COLS <= TMEM_COLS, "scale slots exceed TMEM");
 
 struct alignas(1024) Smem {
   uint8_t a[STAGES][A_BYTES];
   uint8_t b[STAGES][B_BYTES];
-  alignas(128) uint8_t sfa[STAGES][SFA_BYTES];
-  alignas(128) uint8_t sfb[STAGES][SFB_BYTES];
-  uint64_t full[STAGES];     // A/B landed (1 arrival + tx bytes)
-  uint64_t sf_full[STAGES];  // scale factors landed and shuffled (1 arrival from the SF warp)
-  uint64_t empty[STAGES];    // 1 arrival (MMA commit)
-  uint64_t sf_raw[STAGES];   // SF TMA landed (1 arrival + tx)
+  alignas(128) uint8_t sf[STAGES][SFA_BYTES + SFB_BYTES];  // raw row-major scale bytes (TMA)
+  uint64_t full[STAGES];   // A/B bytes + 1 arrival (TMA warp) + SF_WARPS arrivals (scale slot written)
+  uint64_t sf_raw[STAGES]; // raw scale bytes landed (1 arrival + bytes)
+  uint64_t empty[STAGES];  // 1 arrival (MMA commit): the stage's smem and TMEM scale slot are free
   uint64_t tmem_full;
   uint64_t tmem_empty;
   uint64_t mma_done;
@@ -91,23 +97,8 @@ __device__ __forceinline__ Smem& smem_ref(uint8_t* raw) {
   return *reinterpret_cast<Smem*>(p);
 }
 
-// In-place shuffle of one 128-row block of scale bytes (row r at r*16, 16 bytes = 4 MMA steps x 4
-// scales) into 4 consecutive 512-byte blocks, one per MMA step k, where the 16 bytes at l*16 hold
-// the 4 scales of rows l, l+32, l+64, l+96 for that step.  One warp; all reads precede all writes.
-__device__ __forceinline__ void shuffle_sf_block(uint8_t* blk) {
-  const int l = lane_idx();
-  uint4 w[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) w[q] = *reinterpret_cast<const uint4*>(blk + (q * 32 + l) * 16);
-  __syncwarp();
-  uint4 o0 = make_uint4(w[0].x, w[1].x, w[2].x, w[3].x);
-  uint4 o1 = make_uint4(w[0].y, w[1].y, w[2].y, w[3].y);
-  uint4 o2 = make_uint4(w[0].z, w[1].z, w[2].z, w[3].z);
-  uint4 o3 = make_uint4(w[0].w, w[1].w, w[2].w, w[3].w);
-  *reinterpret_cast<uint4*>(blk + 0 * 512 + l * 16) = o0;
-  *reinterpret_cast<uint4*>(blk + 1 * 512 + l * 16) = o1;
-  *reinterpret_cast<uint4*>(blk + 2 * 512 + l * 16) = o2;
-  *reinterpret_cast<uint4*>(blk + 3 * 512 + l * 16) = o3;
+__device__ __forceinline__ uint32_t word(const uint4& v, int k) {
+  return k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
 }
 
 __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __grid_constant__ Nvfp4Params p) {
@@ -121,8 +112,7 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&s.full[i], 1);
-      mbar_init(&s.sf_full[i], 1);
+      mbar_init(&s.full[i], 1 + SF_WARPS);
       mbar_init(&s.empty[i], 1);
       mbar_init(&s.sf_raw[i], 1);
     }
@@ -131,7 +121,7 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
     mbar_init(&s.tmem_empty, EPI_WARPS);
     for (int i = 0; i < Q; ++i) {
       mbar_init(&s.queue.full[i], 1);
-      mbar_init(&s.queue.empty[i], EPI_WARPS + 3);
+      mbar_init(&s.queue.empty[i], EPI_WARPS + 2 + SF_WARPS);
     }
     s.abort = 0;
     fence_mbar_init();
@@ -139,8 +129,6 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
   if (warp == WARP_TMA && lane == 0) {
     tma_prefetch_desc(&p.tmA);
     tma_prefetch_desc(&p.tmB);
-  }
-  if (warp == WARP_SF && lane == 0) {
     tma_prefetch_desc(&p.tmSFA);
     tma_prefetch_desc(&p.tmSFB);
   }
@@ -178,6 +166,9 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
           mbar_arrive_expect_tx(&s.full[pos.stage], A_BYTES + B_BYTES);
           tma_load_2d(s.a[pos.stage], &p.tmA, &s.full[pos.stage], kb * (BK / 2), u.row0);
           tma_load_3d(s.b[pos.stage], &p.tmB, &s.full[pos.stage], kb * (BK / 2), u.n0, u.g);
+          mbar_arrive_expect_tx(&s.sf_raw[pos.stage], SFA_BYTES + SFB_BYTES);
+          tma_load_2d(s.sf[pos.stage], &p.tmSFA, &s.sf_raw[pos.stage], kb * (BK / 16), u.row0);
+          tma_load_3d(s.sf[pos.stage] + SFA_BYTES, &p.tmSFB, &s.sf_raw[pos.stage], kb * (BK / 16), u.n0, u.g);
         }
         __syncwarp();
         ++issued;
@@ -185,6 +176,7 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
       }
     }
     if (ok) {
+      // producer tail: every stage handed out has been consumed before the CTA may retire
       for (int i = 0; i < STAGES; ++i) {
         if (!mbar_wait(&s.empty[pos.stage], pos.phase ^ 1u, wctx.timeout_ns, wctx.abort, wctx.status, kSiteDrain,
                        pos.stage))
@@ -193,62 +185,52 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
       }
     } else {
       drain_inflight_loads<STAGES>(s.full, pos, issued, wctx);
+      drain_inflight_loads<STAGES>(s.sf_raw, pos, issued, wctx);
     }
-  } else if (warp == WARP_SF) {
-    // Issue the scale loads of step i, then shuffle the oldest step once SF_LAG are outstanding (the
-    // TMA latency of the later steps overlaps).  Steps run over all units of the CTA in order.
+  } else if (warp >= WARP_SF0) {
+    // ------------------------------------------------------------------ scale-factor warps
+    // Every quarter receives the same words (the replicated layout): lane l reads raw rows l + 32c.
+    const int qt = warp & 3;
+    const uint32_t lane_addr = static_cast<uint32_t>(qt * 32) << 16;
     int qslot = 0;
     uint32_t qphase = 0;
-    RingPos<STAGES> pos;     // next step to issue
-    RingPos<STAGES> old;     // oldest issued, not yet shuffled
-    long long issued = 0;
-    int pending = 0;
+    RingPos<STAGES> pos;
     bool ok = true;
-    auto process_oldest = [&]() -> bool {
-      if (!mbar_wait(&s.sf_raw[old.stage], old.phase, wctx.timeout_ns, wctx.abort, wctx.status, kSiteSfRaw,
-                     old.stage))
-        return false;
-      shuffle_sf_block(s.sfa[old.stage]);
-      shuffle_sf_block(s.sfb[old.stage]);
-      shuffle_sf_block(s.sfb[old.stage] + 2048);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.sf_full[old.stage]);
-      old.advance();
-      --pending;
-      return true;
-    };
     while (ok) {
       Unit u;
-      if (!queue_pop(s.queue, qslot, qphase, u, wctx)) {
-        ok = false;
-        break;
-      }
+      if (!queue_pop(s.queue, qslot, qphase, u, wctx)) break;
       if (!u.valid) break;
       for (int kb = 0; kb < KS; ++kb) {
-        if (!mbar_wait(&s.empty[pos.stage], pos.phase ^ 1u, wctx.timeout_ns, wctx.abort, wctx.status,
-                       kSiteSmemEmpty, pos.stage)) {
+        // the raw bytes of this use of the stage have landed (they were loaded after the stage was
+        // freed, so the slot's previous MMAs are complete as well)
+        if (!mbar_wait(&s.sf_raw[pos.stage], pos.phase, wctx.timeout_ns, wctx.abort, wctx.status, kSiteSfRaw,
+                       pos.stage)) {
           ok = false;
           break;
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&s.sf_raw[pos.stage], SFA_BYTES + SFB_BYTES);
-          tma_load_2d(s.sfa[pos.stage], &p.tmSFA, &s.sf_raw[pos.stage], kb * (BK / 16), u.row0);
-          tma_load_3d(s.sfb[pos.stage], &p.tmSFB, &s.sf_raw[pos.stage], kb * (BK / 16), u.n0, u.g);
-        }
+        tc_fence_after();
+        const uint4* raw = reinterpret_cast<const uint4*>(s.sf[pos.stage]);
+        uint4 va[4], vb[8];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) va[c] = raw[32 * c + lane];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) vb[c] = raw[BM + 32 * c + lane];
+        uint32_t ra16[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) ra16[j] = word(va[j & 3], j >> 2);
+        uint32_t rb32[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) rb32[j] = word(vb[j & 7], j >> 3);
+        const uint32_t slot = tmem_base + lane_addr + COL_SF0 + static_cast<uint32_t>(pos.stage) * SF_SLOT_COLS;
+        tmem_st_x16(slot, ra16);
+        tmem_st_x32(slot + SFB_OFF, rb32);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
-        ++issued;
+        if (lane == 0) mbar_arrive(&s.full[pos.stage]);
         pos.advance();
-        if (++pending >= SF_LAG && !process_oldest()) {
-          ok = false;
-          break;
-        }
       }
     }
-    while (ok && pending > 0) {
-      if (!process_oldest()) ok = false;
-    }
-    if (!ok) drain_inflight_loads<STAGES>(s.sf_raw, pos, issued, wctx);
   } else if (warp == WARP_MMA) {
     constexpr uint32_t IDESC = idesc_mxf4nvf4(BM, BN);
     int qslot = 0;
@@ -264,8 +246,6 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
       tc_fence_after();
       for (int kb = 0; kb < KS; ++kb) {
         if (!mbar_wait(&s.full[pos.stage], pos.phase, wctx.timeout_ns, wctx.abort, wctx.status, kSiteSmemFull,
-                       pos.stage) ||
-            !mbar_wait(&s.sf_full[pos.stage], pos.phase, wctx.timeout_ns, wctx.abort, wctx.status, kSiteSmemFull,
                        pos.stage)) {
           ok = false;
           break;
@@ -274,18 +254,11 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
         if (lane == 0) {
           const uint64_t da = sdesc_k_sw128(smem_u32(s.a[pos.stage]));
           const uint64_t db = sdesc_k_sw128(smem_u32(s.b[pos.stage]));
-          const uint32_t sfa_s = smem_u32(s.sfa[pos.stage]);
-          const uint32_t sfb_s = smem_u32(s.sfb[pos.stage]);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            tc_cp_32x128b_warpx4(tmem_base + COL_SFA + 4 * k, sdesc_sf(sfa_s + k * 512));
-            tc_cp_32x128b_warpx4(tmem_base + COL_SFB + 8 * k, sdesc_sf(sfb_s + k * 512));
-            tc_cp_32x128b_warpx4(tmem_base + COL_SFB + 8 * k + 4, sdesc_sf(sfb_s + 2048 + k * 512));
-          }
+          const uint32_t sf = tmem_base + COL_SF0 + static_cast<uint32_t>(pos.stage) * SF_SLOT_COLS;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             mma_mxf4nvf4(tmem_base, da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k), IDESC,
-                         tmem_base + COL_SFA + 4 * k, tmem_base + COL_SFB + 8 * k, (kb > 0 || k > 0) ? 1u : 0u);
+                         sf + 4 * k, sf + SFB_OFF + 8 * k, (kb > 0 || k > 0) ? 1u : 0u);
           }
           tc_commit(&s.empty[pos.stage]);
           if (kb == KS - 1) tc_commit(&s.tmem_full);
@@ -314,15 +287,20 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
       if (!mbar_wait(&s.tmem_full, acc_phase, wctx.timeout_ns, wctx.abort, wctx.status, kSiteTmemFull, 0)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + lane_addr + static_cast<uint32_t>(half * 128);
-      uint32_t v[128];
+      uint32_t o[64];  // 128 BF16 values of this row, packed in pairs
 #pragma unroll
-      for (int c = 0; c < 128; c += 16) {
-        uint32_t t[16];
-        tmem_ld_x16(taddr + c, t);
+      for (int c = 0; c < 128; c += 32) {
+        uint32_t v0[16], v1[16];
+        tmem_ld_x16(taddr + c, v0);
+        tmem_ld_x16(taddr + c + 16, v1);
+        tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[c + i] = t[i];
+        for (int i = 0; i < 8; ++i) {
+          o[c / 2 + i] = pack_bf16x2(__uint_as_float(v0[2 * i]) * alpha, __uint_as_float(v0[2 * i + 1]) * alpha);
+          o[c / 2 + 8 + i] =
+              pack_bf16x2(__uint_as_float(v1[2 * i]) * alpha, __uint_as_float(v1[2 * i + 1]) * alpha);
+        }
       }
-      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.tmem_empty);
@@ -334,14 +312,8 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
         __nv_bfloat16* dst = p.C + static_cast<size_t>(row) * p.N + col0;
 #pragma unroll
         for (int c = 0; c < 128; c += 8) {
-          if (c < ncols) {
-            uint4 o;
-            o.x = pack_bf16x2(__uint_as_float(v[c + 0]) * alpha, __uint_as_float(v[c + 1]) * alpha);
-            o.y = pack_bf16x2(__uint_as_float(v[c + 2]) * alpha, __uint_as_float(v[c + 3]) * alpha);
-            o.z = pack_bf16x2(__uint_as_float(v[c + 4]) * alpha, __uint_as_float(v[c + 5]) * alpha);
-            o.w = pack_bf16x2(__uint_as_float(v[c + 6]) * alpha, __uint_as_float(v[c + 7]) * alpha);
-            *reinterpret_cast<uint4*>(dst + c) = o;
-          }
+          if (c < ncols)
+            *reinterpret_cast<uint4*>(dst + c) = make_uint4(o[c / 2], o[c / 2 + 1], o[c / 2 + 2], o[c / 2 + 3]);
         }
       }
     }
