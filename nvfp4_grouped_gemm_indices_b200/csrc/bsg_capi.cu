@@ -52,6 +52,7 @@ struct DeviceState {
   bool fp8_attr = false;
   bool nvfp4_attr = false;
   int fp8_pair_clusters = 0;
+  int nvfp4_pair_clusters = 0;
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -334,6 +335,10 @@ bsg_status bsg_nvfp4_gemm(const void* A, const void* B, const void* sfa, const v
   DeviceState* dev = nullptr;
   if ((st = device_state(&dev)) != BSG_OK) return st;
 
+  // tactic 0: one SM per 128 x 256 tile; tactic 1: an SM pair per 256 x 256 tile (cta_group::2)
+  const int tactic = bsg_choose_tactic(1, M, N, K, G, dev->sm_count);
+  const int cg = tactic == 1 ? 2 : 1;
+
   bsg::Nvfp4Params p;
   memset(&p, 0, sizeof(p));
   const uint64_t Kb = static_cast<uint64_t>(K) / 2;   // packed bytes per row
@@ -348,7 +353,8 @@ bsg_status bsg_nvfp4_gemm(const void* A, const void* B, const void* sfa, const v
   {
     const uint64_t dims[3] = {Kb, static_cast<uint64_t>(N), static_cast<uint64_t>(G)};
     const uint64_t str[2] = {Kb, static_cast<uint64_t>(N) * Kb};
-    const uint32_t box[3] = {128u, static_cast<uint32_t>(bsg::nvfp4::BN), 1u};
+    // B rows per CTA and stage: 256 (one SM) or 128 (each CTA of an SM pair)
+    const uint32_t box[3] = {128u, static_cast<uint32_t>(bsg::nvfp4::BN / cg), 1u};
     const bool oob[3] = {false, true, false};
     if ((st = encode(&p.tmB, "B", B, 3, dims, str, box, oob, CU_TENSOR_MAP_SWIZZLE_128B)) != BSG_OK) return st;
   }
@@ -381,13 +387,54 @@ bsg_status bsg_nvfp4_gemm(const void* A, const void* B, const void* sfa, const v
   cudaError_t e;
   if (!dev->nvfp4_attr) {
     e = cudaFuncSetAttribute(bsg::nvfp4::bsg_nvfp4_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(bsg::nvfp4::SMEM_BYTES));
+                             static_cast<int>(bsg::nvfp4::smem_bytes<1>()));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(nvfp4 kernel smem)");
+    e = cudaFuncSetAttribute(bsg::nvfp4::bsg_nvfp4_grouped_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bsg::nvfp4::smem_bytes<2>()));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(nvfp4 2-SM kernel smem)");
+    cudaLaunchConfig_t qc = {};
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = 2;
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    qc.gridDim = dim3(2 * (dev->sm_count / 2), 1, 1);
+    qc.blockDim = dim3(bsg::nvfp4::THREADS, 1, 1);
+    qc.dynamicSmemBytes = bsg::nvfp4::smem_bytes<2>();
+    qc.attrs = qa;
+    qc.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, bsg::nvfp4::bsg_nvfp4_grouped_2sm_kernel, &qc);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(nvfp4 2-SM kernel)");
+    dev->nvfp4_pair_clusters = clusters;
     dev->nvfp4_attr = true;
   }
-  const int grid = bsg_forced_grid(1, grid_for(dev->sm_count, M, N, G, bsg::nvfp4::BN));
-  bsg::nvfp4::bsg_nvfp4_grouped_kernel<<<grid, bsg::nvfp4::THREADS, bsg::nvfp4::SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(
-      p);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (cg == 1) {
+    const int grid = bsg_forced_grid(1, grid_for(dev->sm_count, M, N, G, bsg::nvfp4::BN));
+    bsg::nvfp4::bsg_nvfp4_grouped_kernel<<<grid, bsg::nvfp4::THREADS, bsg::nvfp4::smem_bytes<1>(), cs>>>(p);
+  } else {
+    if (dev->nvfp4_pair_clusters < 1) return fail(BSG_ERR_CUDA, "no SM-pair cluster fits on this device");
+    const BsgUnitEstimate est = bsg_estimate_units(M, G);
+    const int64_t n_tiles = (N + bsg::nvfp4::BN - 1) / bsg::nvfp4::BN;
+    int64_t clusters = est.pairs * n_tiles;
+    if (clusters > dev->nvfp4_pair_clusters) clusters = dev->nvfp4_pair_clusters;
+    const int grid = 2 * ((bsg_forced_grid(1, static_cast<int>(2 * clusters)) + 1) / 2);
+    cudaLaunchConfig_t lc = {};
+    cudaLaunchAttribute la[1];
+    la[0].id = cudaLaunchAttributeClusterDimension;
+    la[0].val.clusterDim.x = 2;
+    la[0].val.clusterDim.y = 1;
+    la[0].val.clusterDim.z = 1;
+    lc.gridDim = dim3(grid, 1, 1);
+    lc.blockDim = dim3(bsg::nvfp4::THREADS, 1, 1);
+    lc.dynamicSmemBytes = bsg::nvfp4::smem_bytes<2>();
+    lc.stream = cs;
+    lc.attrs = la;
+    lc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&lc, bsg::nvfp4::bsg_nvfp4_grouped_2sm_kernel, p);
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the nvfp4 2-SM kernel");
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launch of the nvfp4 kernel");
   return BSG_OK;

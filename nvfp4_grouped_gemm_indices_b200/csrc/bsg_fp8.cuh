@@ -8,22 +8,19 @@
 // SMs one MMA spans:
 //   CG = 1  a work unit is a 128-row window segment x 256 columns on one SM; two 256-column TMEM
 //           accumulators ping-pong between the MMAs and the promotion.
-//   CG = 2  a cluster of two CTAs on an SM pair computes a 256 x 128 tile with 2-SM tcgen05 MMAs
-//           (cta_group::2): each CTA holds the 128 rows of its own window segment and 64 of the 128
-//           B rows; the even CTA issues the MMAs for both.  Per SM and FLOP this moves the same
-//           bytes through L2 and shared memory as the one-SM 128 x 256 tile, but an accumulator is
-//           only 128 columns wide, so FOUR fit in TMEM: the tensor cores can run three K blocks
-//           ahead of the promotion instead of one, which hides the commit -> promote -> release
-//           hand-off latency (measured ~700 cycles against a 512-cycle MMA block).
+//   CG = 2  a cluster of two CTAs on an SM pair computes a 256 x 256 tile with 2-SM tcgen05 MMAs
+//           (cta_group::2): each CTA holds the 128 rows of its own window segment and 128 of the
+//           256 B rows; the even CTA issues the MMAs for both.  Per SM and K block this moves 32 KB
+//           of A/B through shared memory instead of 48 KB (the MMA reads each CTA's B half once for
+//           both SMs); each CTA promotes its own 128 x 256 partials in two ping-pong accumulators.
 // Roles:
 //   warp 0      producer: TMA of the A box [128 rows x 128 B] and this CTA's B box [BN/CG rows x
 //               128 B] into a STAGES-deep shared-memory ring; the arrival bytes of both CTAs of a
 //               pair count on the even CTA's full barrier.
 //   warp 1      TMEM allocator + (even CTA) single-thread tcgen05.mma issuer: per 128-K block, 4 K steps
-//               of kind::f8f6f4 MMAs into a fresh FP32 accumulator: one 128 x 256 MMA per step (CG 1,
-//               two accumulators of 256 columns that ping-pong), or two 256 x 128 MMAs per step, one
-//               per N half (CG 2, each half with its own two 128-column accumulators), so the tensor
-//               cores run ahead of the epilogue that promotes the previous block.  Completion is
+//               of kind::f8f6f4 MMAs (128 x 256 per step, or 256 x 256 across the pair) into a fresh
+//               FP32 accumulator; two 256-column accumulators ping-pong so the tensor cores run one
+//               block ahead of the epilogue that promotes the previous block.  Completion is
 //               committed to the barriers of both CTAs.
 //   warp 2      scheduler (bsg_sched.cuh): window segmentation, pairing, unit hand-out.
 //   warp 3      scale producer: cp.async of each K block's scales (a_scale of the 128 rows, b_scale
@@ -76,12 +73,12 @@ constexpr int TMEM_COLS = 512;
 
 template <int CG>
 struct Cfg {
-  static constexpr int BN = CG == 1 ? 256 : 128;          // output columns per unit
-  static constexpr int ACC = TMEM_COLS / BN;              // TMEM accumulators: 2 (CG 1) / 4 (CG 2)
+  static constexpr int BN = 256;                         // output columns per unit
+  static constexpr int ACC = TMEM_COLS / BN;              // two TMEM accumulators
   static constexpr int B_BOX_ROWS = BN / CG;              // B rows this CTA loads per stage
   static constexpr int A_BYTES = BM * BK;                 // 16 KB
-  static constexpr int B_BYTES = B_BOX_ROWS * BK;         // 32 KB (CG 1) / 8 KB (CG 2)
-  static constexpr int STAGES = CG == 1 ? 4 : 8;          // 192 KB of ring either way
+  static constexpr int B_BYTES = B_BOX_ROWS * BK;         // 32 KB (CG 1) / 16 KB (CG 2)
+  static constexpr int STAGES = CG == 1 ? 4 : 6;          // 192 KB of ring either way
   static constexpr uint32_t STAGE_TX = CG * (A_BYTES + B_BYTES);  // bytes counted on the even CTA
   static constexpr int EPI_COLS = BN / 4;                 // columns per epilogue warp: 64 / 32
   static constexpr int NB_TILE = BN / 128;                // 128-column scale blocks per tile

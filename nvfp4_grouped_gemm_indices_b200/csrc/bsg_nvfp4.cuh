@@ -4,7 +4,14 @@
 // (SM120+)에서 NVFP4 QMoE를 위한 네이티브 FP4xFP4 Prefill 최적화", section 1:
 //   C[m, n] = bf16( alpha[g] * sum_j sfa[m, j] * sfb[g, n, j] * (A[m, block j] . B[g, n, block j]) )
 //
-// Design (persistent, warp-specialised, one CTA per SM):
+// Design (persistent, warp-specialised, one CTA per SM), templated on CG, the number of SMs one MMA
+// spans:
+//   CG = 1  a work unit is a 128-row window segment x 256 columns on one SM.
+//   CG = 2  a cluster of two CTAs on an SM pair computes a 256 x 256 tile with 2-SM MMAs
+//           (cta_group::2): each CTA holds the 128 rows of its own window segment and 128 of the 256
+//           B rows (so each SM moves 32 KB of A/B per stage through shared memory instead of 48 KB)
+//           and its own scale slots (SFA of its rows, SFB of all 256 columns); the even CTA issues
+//           the MMAs and commits to both CTAs' barriers.
 //   warps 0..7   epilogue: after the last K stage of a unit, read the 128 x BN FP32 accumulator from
 //                TMEM (warp w: lanes 32*(w%4).., columns 128*(w/4)..), scale by alpha[g] and pack to
 //                BF16 while reading, release the accumulator, then store the segment's rows.
@@ -54,10 +61,9 @@ struct Nvfp4Params {
 
 namespace nvfp4 {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;                  // rows per CTA
+constexpr int BN = 256;                  // output columns per unit (both variants)
 constexpr int BK = 256;                  // K elements per stage (128 packed bytes)
-constexpr int STAGES = 4;
 constexpr int Q = 4;
 constexpr int EPI_WARPS = 8;
 constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_SCHED = 10, WARP_SF0 = 11;
@@ -65,60 +71,77 @@ constexpr int SF_WARPS = 4;
 constexpr int NUM_WARPS = WARP_SF0 + SF_WARPS;
 constexpr int THREADS = NUM_WARPS * 32;
 constexpr int A_BYTES = BM * BK / 2;     // 16 KB
-constexpr int B_BYTES = BN * BK / 2;     // 32 KB
 constexpr int SFA_BYTES = BM * BK / 16;  // 2 KB
-constexpr int SFB_BYTES = BN * BK / 16;  // 4 KB
+constexpr int SFB_BYTES = BN * BK / 16;  // 4 KB (every CTA holds the scales of all BN columns)
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t COL_SF0 = 256;        // first scale slot
 constexpr uint32_t SF_SLOT_COLS = 48;    // 16 SFA + 32 SFB columns per stage
 constexpr uint32_t SFB_OFF = 16;
-static_assert(COL_SF0 + STAGES * SF_SLOT_COLS <= TMEM_COLS, "scale slots exceed TMEM");
 
+template <int CG>
+struct Cfg {
+  static constexpr int B_BOX_ROWS = BN / CG;                       // B rows this CTA loads per stage
+  static constexpr int B_BYTES = B_BOX_ROWS * BK / 2;              // 32 KB (CG 1) / 16 KB (CG 2)
+  static constexpr int STAGES = CG == 1 ? 4 : 5;                   // 216 KB / 190 KB of ring
+  static constexpr uint32_t STAGE_TX = CG * (A_BYTES + B_BYTES);   // A/B bytes counted on the even CTA
+  static constexpr int FULL_ARRIVALS = 1 + CG * SF_WARPS;          // TMA warp + every CTA's scale warps
+  static_assert(COL_SF0 + STAGES * SF_SLOT_COLS <= TMEM_COLS, "scale slots exceed TMEM");
+};
+
+template <int CG>
 struct alignas(1024) Smem {
-  uint8_t a[STAGES][A_BYTES];
-  uint8_t b[STAGES][B_BYTES];
-  alignas(128) uint8_t sf[STAGES][SFA_BYTES + SFB_BYTES];  // raw row-major scale bytes (TMA)
-  uint64_t full[STAGES];   // A/B bytes + 1 arrival (TMA warp) + SF_WARPS arrivals (scale slot written)
-  uint64_t sf_raw[STAGES]; // raw scale bytes landed (1 arrival + bytes)
-  uint64_t empty[STAGES];  // 1 arrival (MMA commit): the stage's smem and TMEM scale slot are free
+  uint8_t a[Cfg<CG>::STAGES][A_BYTES];
+  uint8_t b[Cfg<CG>::STAGES][Cfg<CG>::B_BYTES];
+  alignas(128) uint8_t sf[Cfg<CG>::STAGES][SFA_BYTES + SFB_BYTES];  // raw row-major scale bytes (TMA)
+  uint64_t full[Cfg<CG>::STAGES];    // (even CTA) A/B bytes + FULL_ARRIVALS arrivals
+  uint64_t sf_raw[Cfg<CG>::STAGES];  // this CTA's raw scale bytes landed (1 arrival + bytes)
+  uint64_t empty[Cfg<CG>::STAGES];   // 1 MMA commit: the stage's smem and TMEM scale slot are free
   uint64_t tmem_full;
-  uint64_t tmem_empty;
+  uint64_t tmem_empty;               // (even CTA) CG * EPI_WARPS arrivals
   uint64_t mma_done;
   UnitQueue<Q> queue;
   uint32_t tmem_base;
   int abort;
 };
 
-constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;
+template <int CG>
+constexpr size_t smem_bytes() {
+  return sizeof(Smem<CG>) + 1024;  // + alignment slack
+}
 
-__device__ __forceinline__ Smem& smem_ref(uint8_t* raw) {
+template <int CG>
+__device__ __forceinline__ Smem<CG>& smem_ref(uint8_t* raw) {
   uintptr_t p = reinterpret_cast<uintptr_t>(raw);
   p = (p + 1023) & ~static_cast<uintptr_t>(1023);
-  return *reinterpret_cast<Smem*>(p);
+  return *reinterpret_cast<Smem<CG>*>(p);
 }
 
 __device__ __forceinline__ uint32_t word(const uint4& v, int k) {
   return k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
 }
 
-__global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __grid_constant__ Nvfp4Params p) {
+template <int CG>
+__device__ __forceinline__ void nvfp4_kernel_body(const Nvfp4Params& p) {
+  using C = Cfg<CG>;
+  constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
-  Smem& s = smem_ref(smem_raw);
+  Smem<CG>& s = smem_ref<CG>(smem_raw);
   const int warp = warp_idx();
   const int lane = lane_idx();
   const int KS = p.K / BK;
   const int n_tiles = (p.N + BN - 1) / BN;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;   // 0 = the CTA that issues the MMAs
   WaitCtx wctx{p.timeout_ns, &s.abort, p.status};
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&s.full[i], 1 + SF_WARPS);
+      mbar_init(&s.full[i], C::FULL_ARRIVALS);
       mbar_init(&s.empty[i], 1);
       mbar_init(&s.sf_raw[i], 1);
     }
     mbar_init(&s.mma_done, 1);
     mbar_init(&s.tmem_full, 1);
-    mbar_init(&s.tmem_empty, EPI_WARPS);
+    mbar_init(&s.tmem_empty, CG * EPI_WARPS);
     for (int i = 0; i < Q; ++i) {
       mbar_init(&s.queue.full[i], 1);
       mbar_init(&s.queue.empty[i], EPI_WARPS + 2 + SF_WARPS);
@@ -133,16 +156,25 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
     tma_prefetch_desc(&p.tmSFB);
   }
   if (warp == WARP_MMA) {
-    tmem_alloc(&s.tmem_base, TMEM_COLS);
-    tmem_relinquish();
+    if (CG == 2) {
+      tmem_alloc_pair(&s.tmem_base, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&s.tmem_base, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2) {
+    cluster_sync();  // both CTAs' barriers are initialised before either touches the other's
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   const uint32_t tmem_base = s.tmem_base;
 
   if (warp == WARP_SCHED) {
-    run_scheduler<Q, BN, false>(s.queue, p.m_indices, p.M, p.G, n_tiles, p.n_group, wctx, p.debug_mode);
+    run_scheduler<Q, BN, CG == 2>(s.queue, p.m_indices, p.M, p.G, n_tiles, p.n_group, wctx, p.debug_mode);
   } else if (warp == WARP_TMA) {
     int qslot = 0;
     uint32_t qphase = 0;
@@ -163,9 +195,20 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
           break;
         }
         if (lane == 0) {
-          mbar_arrive_expect_tx(&s.full[pos.stage], A_BYTES + B_BYTES);
-          tma_load_2d(s.a[pos.stage], &p.tmA, &s.full[pos.stage], kb * (BK / 2), u.row0);
-          tma_load_3d(s.b[pos.stage], &p.tmB, &s.full[pos.stage], kb * (BK / 2), u.n0, u.g);
+          if (CG == 1) {
+            mbar_arrive_expect_tx(&s.full[pos.stage], C::STAGE_TX);
+            tma_load_2d(s.a[pos.stage], &p.tmA, &s.full[pos.stage], kb * (BK / 2), u.row0);
+            tma_load_3d(s.b[pos.stage], &p.tmB, &s.full[pos.stage], kb * (BK / 2), u.n0, u.g);
+          } else {
+            // A/B bytes of both CTAs count on the even CTA's full barrier; this CTA's B box is rows
+            // n0 + rank * 128 of expert g
+            const uint32_t leader_full = mapa_shared(smem_u32(&s.full[pos.stage]), 0);
+            if (rank == 0) mbar_arrive_expect_tx(&s.full[pos.stage], C::STAGE_TX);
+            tma_load_2d_pair(s.a[pos.stage], &p.tmA, leader_full, kb * (BK / 2), u.row0);
+            tma_load_3d_pair(s.b[pos.stage], &p.tmB, leader_full, kb * (BK / 2),
+                             u.n0 + static_cast<int>(rank) * C::B_BOX_ROWS, u.g);
+          }
+          // this CTA's own scale bytes (SFA of its rows, SFB of all BN columns) on its own barrier
           mbar_arrive_expect_tx(&s.sf_raw[pos.stage], SFA_BYTES + SFB_BYTES);
           tma_load_2d(s.sf[pos.stage], &p.tmSFA, &s.sf_raw[pos.stage], kb * (BK / 16), u.row0);
           tma_load_3d(s.sf[pos.stage] + SFA_BYTES, &p.tmSFB, &s.sf_raw[pos.stage], kb * (BK / 16), u.n0, u.g);
@@ -184,7 +227,9 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
         pos.advance();
       }
     } else {
-      drain_inflight_loads<STAGES>(s.full, pos, issued, wctx);
+      // (CG 2: the odd CTA's A/B loads land on the even CTA's barrier; the closing cluster barrier
+      // keeps this CTA's shared memory alive until the even CTA has drained those too.)
+      if (CG == 1 || rank == 0) drain_inflight_loads<STAGES>(s.full, pos, issued, wctx);
       drain_inflight_loads<STAGES>(s.sf_raw, pos, issued, wctx);
     }
   } else if (warp >= WARP_SF0) {
@@ -227,12 +272,17 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s.full[pos.stage]);
+        if (lane == 0) {
+          if (CG == 1 || rank == 0)
+            mbar_arrive(&s.full[pos.stage]);
+          else
+            mbar_arrive_cluster(mapa_shared(smem_u32(&s.full[pos.stage]), 0));
+        }
         pos.advance();
       }
     }
   } else if (warp == WARP_MMA) {
-    constexpr uint32_t IDESC = idesc_mxf4nvf4(BM, BN);
+    constexpr uint32_t IDESC = idesc_mxf4nvf4(BM * CG, BN);
     int qslot = 0;
     uint32_t qphase = 0;
     RingPos<STAGES> pos;
@@ -241,6 +291,7 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
     while (ok) {
       Unit u;
       if (!queue_pop(s.queue, qslot, qphase, u, wctx) || !u.valid) break;
+      if (CG == 2 && rank != 0) continue;  // the even CTA issues the pair's MMAs
       if (!mbar_wait(&s.tmem_empty, acc_phase ^ 1u, wctx.timeout_ns, wctx.abort, wctx.status, kSiteTmemEmpty, 0))
         break;
       tc_fence_after();
@@ -257,20 +308,38 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
           const uint32_t sf = tmem_base + COL_SF0 + static_cast<uint32_t>(pos.stage) * SF_SLOT_COLS;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            mma_mxf4nvf4(tmem_base, da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k), IDESC,
-                         sf + 4 * k, sf + SFB_OFF + 8 * k, (kb > 0 || k > 0) ? 1u : 0u);
+            const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+            if (CG == 1)
+              mma_mxf4nvf4(tmem_base, da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k), IDESC,
+                           sf + 4 * k, sf + SFB_OFF + 8 * k, acc);
+            else
+              mma_mxf4nvf4_pair(tmem_base, da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k),
+                                IDESC, sf + 4 * k, sf + SFB_OFF + 8 * k, acc);
           }
-          tc_commit(&s.empty[pos.stage]);
-          if (kb == KS - 1) tc_commit(&s.tmem_full);
+          if (CG == 1) {
+            tc_commit(&s.empty[pos.stage]);
+            if (kb == KS - 1) tc_commit(&s.tmem_full);
+          } else {
+            tc_commit_pair_multicast(&s.empty[pos.stage], 0x3);
+            if (kb == KS - 1) tc_commit_pair_multicast(&s.tmem_full, 0x3);
+          }
         }
         __syncwarp();
         pos.advance();
       }
       acc_phase ^= 1u;
     }
-    if (lane == 0) tc_commit(&s.mma_done);
-    __syncwarp();
-    mbar_wait(&s.mma_done, 0, wctx.timeout_ns, nullptr, nullptr, kSiteDrain, 0);
+    // every MMA this thread issued has completed before TMEM may be released
+    if (CG == 1 || rank == 0) {
+      if (lane == 0) {
+        if (CG == 1)
+          tc_commit(&s.mma_done);
+        else
+          tc_commit_pair_multicast(&s.mma_done, 0x1);
+      }
+      __syncwarp();
+      mbar_wait(&s.mma_done, 0, wctx.timeout_ns, nullptr, nullptr, kSiteDrain, 0);
+    }
   } else {
     // ------------------------------------------------------------------ epilogue warps 0..7
     const int quarter = warp & 3;
@@ -303,7 +372,12 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s.tmem_empty);
+      if (lane == 0) {
+        if (CG == 1 || rank == 0)
+          mbar_arrive(&s.tmem_empty);
+        else
+          mbar_arrive_cluster(mapa_shared(smem_u32(&s.tmem_empty), 0));
+      }
       acc_phase ^= 1u;
       const int row = u.row0 + r;
       const int col0 = u.n0 + half * 128;
@@ -320,9 +394,27 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __g
   }
 
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2) {
+    cluster_sync();  // the even CTA's MMAs into the odd CTA's TMEM are complete (mma_done waited)
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
-  if (warp == WARP_MMA) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == WARP_MMA) {
+    if (CG == 2)
+      tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_kernel(const __grid_constant__ Nvfp4Params p) {
+  nvfp4_kernel_body<1>(p);
+}
+
+// Launched as clusters of 2 CTAs (grid a multiple of 2).
+__global__ void __launch_bounds__(THREADS, 1) bsg_nvfp4_grouped_2sm_kernel(const __grid_constant__ Nvfp4Params p) {
+  nvfp4_kernel_body<2>(p);
 }
 
 }  // namespace nvfp4

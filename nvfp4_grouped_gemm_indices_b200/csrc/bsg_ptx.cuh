@@ -288,8 +288,10 @@ __device__ __forceinline__ void cluster_sync() {
 }
 
 // Arrival on an mbarrier of another CTA of the cluster (address from mapa_shared).  CTA-scope
-// release: the arrival only publishes that this thread's tcgen05 reads (ordered before it by
-// tcgen05.fence::before_thread_sync) are done; a cluster-scope release would fence every arrival.
+// release: the arrival publishes that this thread's tcgen05 loads or stores (completed by
+// tcgen05.wait::ld / wait::st and ordered before it by tcgen05.fence::before_thread_sync) are done.
+// A cluster-scope release fences every arrival and, on the critical path of the NVFP4 pair kernel's
+// scale slots, halved its throughput.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
@@ -336,6 +338,19 @@ __device__ __forceinline__ void mma_f8f6f4_pair(uint32_t d_tmem, uint64_t a_desc
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 2-SM block-scaled FP4 MMA (issued by the even CTA): as mma_f8f6f4_pair, with each CTA's scale
+// factors read from its own TMEM at the given columns.
+__device__ __forceinline__ void mma_mxf4nvf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
       : "memory");
 }
 

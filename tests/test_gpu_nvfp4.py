@@ -15,6 +15,17 @@ from gpu_util import (SENTINEL, DevWorkload, bits, compare, oracle_rows, routed_
 
 pytestmark = pytest.mark.gpu
 
+NVFP4_TACTICS = [0, 1]  # 0: one SM per 128 x 256 tile; 1: an SM pair per 256 x 256 tile (cta_group::2)
+
+
+@pytest.fixture(params=NVFP4_TACTICS, ids=lambda t: f"tactic{t}", autouse=True)
+def tactic(request):
+    if request.param >= bsg.bsg_num_tactics(1):
+        pytest.skip("tactic not built")
+    bsg.bsg_set_tactic(1, request.param)
+    yield request.param
+    bsg.bsg_set_tactic(1, -1)
+
 
 def full_check(w):
     d = DevWorkload(w)
