@@ -219,6 +219,13 @@ class Runner:
             self.s1, self.s2, self.s3 = dev(w.sfa), dev(w.sfb), dev(w.alpha)
         self.C = torch.zeros((w.M, w.N), dtype=torch.bfloat16, device="cuda")
 
+    def tactic(self):
+        """Name of the tactic the library's chooser picks for this workload."""
+        w = self.w
+        kind = 0 if w.kind == "fp8" else 1
+        sms = torch_sm_count()
+        return self.bsg.bsg_tactic_name(kind, self.bsg.bsg_choose_tactic(kind, w.M, w.N, w.K, w.G, sms))
+
     def launch(self, stream, A=None, B=None, s1=None, s2=None, s3=None, idx=None, C=None):
         w = self.w
         A = self.A if A is None else A
@@ -232,6 +239,11 @@ class Runner:
             self.bsg.bsg_fp8_grouped_gemm(A, B, s1, s2, idx, C, w.M, w.N, w.K, w.G, stream)
         else:
             self.bsg.bsg_nvfp4_gemm(A, B, s1, s2, s3, idx, C, w.M, w.N, w.K, w.G, stream)
+
+
+def torch_sm_count():
+    import torch
+    return torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
 
 
 def time_kernel(runner, steps, warmup, flush=None):
@@ -328,8 +340,10 @@ def roofline(w, per_launch_s, peaks, peak_src, sustained=False):
                 "frac": round(ach / hbm, 4), "traffic": traffic, "algorithmic_bytes": nbytes,
                 "peak_source": f"{peak_src} hbm_gbs (STREAM-style copy)"}
     ach = flops / per_launch_s / 1e12
+    sustained_peak = peaks["bf16_tflops_sustained"] * DTYPE_RATIO[w.kind]
     return {"bound": "tensor", "achieved": round(ach, 1), "peak": round(tensor_peak, 1), "unit": "TFLOP/s",
-            "frac": round(ach / tensor_peak, 4), "traffic": traffic, "algorithmic_bytes": nbytes,
+            "frac": round(ach / tensor_peak, 4), "frac_of_sustained_peak": round(ach / sustained_peak, 4),
+            "traffic": traffic, "algorithmic_bytes": nbytes,
             "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} x {DTYPE_RATIO[w.kind]:g} "
                            f"({w.kind} : bf16 nominal dense ratio)"}
 
@@ -417,7 +431,7 @@ def run_bsg(args):
         "dtype": "e4m3xe4m3->f32 (fp32 per-128 scales), bf16 out" if w.kind == "fp8"
         else "e2m1xe2m1 (ue4m3 per-16 scales)->f32, bf16 out",
         "data": "synthetic (seeded; quantised N(0,1) activations, N(0,0.02) / N(0,1) weights)",
-        "config": config_desc(w, args.config, flush),
+        "config": dict(config_desc(w, args.config, flush), tactic=r.tactic()),
         "roofline": roofline(w, per, peaks, peak_src),
         "gpu_launches": args.steps,
         "clocks": clocks,
@@ -441,7 +455,8 @@ def run_bsg(args):
                 steps = max(20, min(args.steps, 200))
                 tot, pl = time_kernel(r, steps, max(3, args.warmup // 4), fl)
                 rf = roofline(wc, pl, peaks, peak_src)
-                also[wc.name] = {"tflops": round(wc.flops / pl / 1e12, 2), "us_per_launch": round(pl * 1e6, 2),
+                also[wc.name] = {"tactic": r.tactic(), "tflops": round(wc.flops / pl / 1e12, 2),
+                                 "us_per_launch": round(pl * 1e6, 2),
                                  "roofline": rf, "l2": "flushed" if fl else "inputs > L2"}
             line["also"] = also
     if rank == 0:
