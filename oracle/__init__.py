@@ -15,6 +15,9 @@ Functions (all numpy in, numpy out):
   per-expert FP32 ``alpha``.
 * ``window_plan(m_indices, M, G)`` -- the window segmentation the pages describe (same FP8 page,
   section 2): maximal equal runs of routed rows cut at 128-row window edges.
+* ``enc_e4m3``, ``enc_e2m1``, ``quant_fp8_rows``, ``quant_nvfp4_rows`` -- the step before the GEMM:
+  BF16 activations (optionally gathered by a row map, the MoE expand) quantised into the GEMM's
+  input formats, from the format definitions (RNE, saturating) with every step in IEEE fp32.
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py`` (decode tables, exact
 integer grids, grouped == dense, exact rational brute force, fp64 library matmul, the printed CTA
@@ -47,6 +50,14 @@ def lib():
         L.bsg_oracle_fp8_grouped.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, i64, p, p]
         L.bsg_oracle_nvfp4.restype = ctypes.c_int
         L.bsg_oracle_nvfp4.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, p, i64, p, p]
+        L.bsg_oracle_enc_e4m3.restype = ctypes.c_uint8
+        L.bsg_oracle_enc_e4m3.argtypes = [ctypes.c_float]
+        L.bsg_oracle_enc_e2m1.restype = ctypes.c_uint8
+        L.bsg_oracle_enc_e2m1.argtypes = [ctypes.c_float]
+        L.bsg_oracle_quant_fp8_rows.restype = ctypes.c_int
+        L.bsg_oracle_quant_fp8_rows.argtypes = [p, p, i64, i64, i64, p, p]
+        L.bsg_oracle_quant_nvfp4_rows.restype = ctypes.c_int
+        L.bsg_oracle_quant_nvfp4_rows.argtypes = [p, p, ctypes.c_float, i64, i64, i64, p, p]
         L.bsg_oracle_max_threads.restype = ctypes.c_int
         L.bsg_oracle_set_threads.argtypes = [ctypes.c_int]
         _lib = L
@@ -127,6 +138,59 @@ def nvfp4(A, B, sfa, sfb, alpha, m_indices, M, N, K, G, rows=None, out_bf16=None
     if rc != 0:
         raise ValueError("oracle nvfp4: invalid sizes")
     return out_bf16, f64
+
+
+def enc_e4m3(x):
+    """fp32 value(s) -> E4M3 code(s): round to nearest even, saturating at +-448."""
+    L = lib()
+    a = np.asarray(x, dtype=np.float32)
+    return np.array([L.bsg_oracle_enc_e4m3(float(v)) for v in a.ravel()], dtype=np.uint8).reshape(a.shape)
+
+
+def enc_e2m1(x):
+    """fp32 value(s) -> E2M1 code(s) 0..15: round to nearest even, saturating at +-6."""
+    L = lib()
+    a = np.asarray(x, dtype=np.float32)
+    return np.array([L.bsg_oracle_enc_e2m1(float(v)) for v in a.ravel()], dtype=np.uint8).reshape(a.shape)
+
+
+def quant_fp8_rows(X_bf16_bits, M=None, src_rows=None, A=None, scale=None):
+    """Activation quantisation to the FP8 GEMM's A operand: per 1 x 128 block, scale = amax/448,
+    code = e4m3_rne_satfinite(x / scale) in fp32.  X: uint16 bf16 bits [M_in, K]; output row m is
+    input row src_rows[m] (or m).  Returns (A uint8 [M, K], scale f32 [M, K/128]); rows whose
+    source is out of range keep the initial contents of A / scale (default 0xFF / NaN)."""
+    L = lib()
+    X = np.ascontiguousarray(X_bf16_bits, dtype=np.uint16)
+    M_in, K = X.shape
+    M = M_in if M is None else int(M)
+    src = None if src_rows is None else np.ascontiguousarray(src_rows, dtype=np.int32)
+    if A is None:
+        A = np.full((M, K), 0xFF, dtype=np.uint8)
+    if scale is None:
+        scale = np.full((M, K // 128), np.nan, dtype=np.float32)
+    rc = L.bsg_oracle_quant_fp8_rows(_ptr(X), _ptr(src), M_in, M, K, _ptr(A), _ptr(scale))
+    if rc != 0:
+        raise ValueError("oracle quant_fp8_rows: invalid sizes")
+    return A, scale
+
+
+def quant_nvfp4_rows(X_bf16_bits, gs, M=None, src_rows=None, A=None, sf=None):
+    """Activation quantisation to the NVFP4 GEMM's A operand with global scale gs: per 1 x 16
+    block, s = ue4m3_rne_satfinite((amax/6)/gs), code = e2m1_rne_satfinite(x / (dec(s) * gs)), all in
+    fp32.  Returns (A uint8 [M, K/2] packed, low nibble = lower K; sf uint8 [M, K/16])."""
+    L = lib()
+    X = np.ascontiguousarray(X_bf16_bits, dtype=np.uint16)
+    M_in, K = X.shape
+    M = M_in if M is None else int(M)
+    src = None if src_rows is None else np.ascontiguousarray(src_rows, dtype=np.int32)
+    if A is None:
+        A = np.full((M, K // 2), 0xFF, dtype=np.uint8)
+    if sf is None:
+        sf = np.full((M, K // 16), 0xFF, dtype=np.uint8)
+    rc = L.bsg_oracle_quant_nvfp4_rows(_ptr(X), _ptr(src), float(np.float32(gs)), M_in, M, K, _ptr(A), _ptr(sf))
+    if rc != 0:
+        raise ValueError("oracle quant_nvfp4_rows: invalid sizes")
+    return A, sf
 
 
 def set_threads(n):

@@ -197,6 +197,133 @@ int bsg_oracle_nvfp4(const uint8_t* A, const uint8_t* B, const uint8_t* sfa, con
   return 0;
 }
 
+/* ---------------------------------------------------------------- activation quantisers ---- */
+
+/*
+ * The step just before the GEMM: BF16 activations quantised per row block into the GEMM's input
+ * formats, optionally gathering the rows first (the MoE "expand" that puts each expert's tokens in
+ * contiguous runs; row m of the output is row src_rows[m] of the input).  Written from the format
+ * definitions and the quantisation recipe of the two GEMMs' inputs:
+ *
+ *   FP8, per 1 x 128 block:  scale = amax / 448;  code = e4m3_rne_satfinite(x / scale)
+ *   NVFP4, per 1 x 16 block, global scale gs:
+ *       s = ue4m3_rne_satfinite((amax16 / 6) / gs);  code = e2m1_rne_satfinite(x / (dec(s) * gs))
+ *
+ * Every operation is the IEEE fp32 one (division and multiplication correctly rounded, no fused
+ * multiply-add), because the quantised code is an integer decided in fp32 on the GPU as well.  A
+ * block whose scale is zero gets all-zero codes.  The encoders round to the nearest representable
+ * value, ties to the even code, and saturate at the largest finite magnitude (448, 6).
+ */
+
+/* fp32 -> E4M3 (FN) code: RNE, saturating at +-448; NaN -> 0x7F with the sign. */
+uint8_t bsg_oracle_enc_e4m3(float x) {
+  uint8_t sign = signbit(x) ? 0x80u : 0u;
+  double a = fabs((double)x);
+  if (isnan(x)) return (uint8_t)(sign | 0x7Fu);
+  if (a >= 448.0) return (uint8_t)(sign | 0x7Eu);
+  if (a < ldexp(1.0, -6)) {
+    /* subnormal spacing 2^-9; a result of 8 quanta is the smallest normal, code 0x08 */
+    double r = nearbyint(a / ldexp(1.0, -9));
+    return (uint8_t)(sign | (uint8_t)r);
+  }
+  int e2;
+  frexp(a, &e2);                         /* a in [2^(e2-1), 2^e2) */
+  int e = e2 - 1;
+  double r = nearbyint(a / ldexp(1.0, e - 3)); /* 8..16 quanta of the binade */
+  int code = (e + 6) * 8 + (int)r;       /* (e + 7) << 3 | (r - 8); r = 16 carries into the exponent */
+  if (code > 0x7E) code = 0x7E;
+  return (uint8_t)(sign | (uint8_t)code);
+}
+
+/* fp32 -> E2M1 code (0..15): RNE on the magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}, saturating at +-6. */
+uint8_t bsg_oracle_enc_e2m1(float x) {
+  uint8_t sign = signbit(x) ? 0x8u : 0u;
+  double a = fabs((double)x);
+  int code;
+  if (a >= 6.0) {
+    code = 7;
+  } else if (a < 2.0) {
+    code = (int)nearbyint(a / 0.5);      /* quantum 0.5: codes 0..4 */
+  } else if (a < 4.0) {
+    code = 2 + (int)nearbyint(a);        /* quantum 1: codes 4..6 */
+  } else {
+    code = 4 + (int)nearbyint(a / 2.0);  /* quantum 2: codes 6..7 */
+  }
+  return (uint8_t)(sign | (uint8_t)code);
+}
+
+static float bf16_bits_to_f32(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, sizeof(f));
+  return f;
+}
+
+/* X bf16 bits [M_in, K]; src_rows int32 [M] or NULL (output row m = input row m, M_in >= M).
+ * A uint8 [M, K] E4M3 codes; scale f32 [M, K/128].  Output rows whose source is outside
+ * [0, M_in) are left untouched.  Returns 0, or -1 for an invalid size. */
+int bsg_oracle_quant_fp8_rows(const uint16_t* X, const int32_t* src_rows, int64_t M_in, int64_t M, int64_t K,
+                              uint8_t* A, float* scale) {
+  if (M < 0 || M_in < 0 || K <= 0 || K % 128 != 0) return -1;
+  const int64_t KB = K / 128;
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    int64_t src = src_rows ? (int64_t)src_rows[m] : m;
+    if (src < 0 || src >= M_in) continue;
+    const uint16_t* x = X + src * K;
+    for (int64_t kb = 0; kb < KB; ++kb) {
+      float amax = 0.0f;
+      for (int64_t k = 0; k < 128; ++k) {
+        float v = fabsf(bf16_bits_to_f32(x[kb * 128 + k]));
+        if (v > amax) amax = v;
+      }
+      volatile float s = amax / 448.0f;
+      scale[m * KB + kb] = s;
+      for (int64_t k = 0; k < 128; ++k) {
+        float v = bf16_bits_to_f32(x[kb * 128 + k]);
+        volatile float q = (s > 0.0f) ? v / s : 0.0f;
+        A[m * K + kb * 128 + k] = bsg_oracle_enc_e4m3(q);
+      }
+    }
+  }
+  return 0;
+}
+
+/* X bf16 bits [M_in, K]; gs the global scale (> 0); A uint8 [M, K/2] packed E2M1 (lower-K element
+ * in the low nibble); sf uint8 [M, K/16] UE4M3 codes.  src_rows as above.  Returns 0 or -1. */
+int bsg_oracle_quant_nvfp4_rows(const uint16_t* X, const int32_t* src_rows, float gs, int64_t M_in, int64_t M,
+                                int64_t K, uint8_t* A, uint8_t* sf) {
+  if (M < 0 || M_in < 0 || K <= 0 || K % 16 != 0) return -1;
+  const int64_t KS = K / 16;
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    int64_t src = src_rows ? (int64_t)src_rows[m] : m;
+    if (src < 0 || src >= M_in) continue;
+    const uint16_t* x = X + src * K;
+    for (int64_t j = 0; j < KS; ++j) {
+      float amax = 0.0f;
+      for (int64_t k = 0; k < 16; ++k) {
+        float v = fabsf(bf16_bits_to_f32(x[j * 16 + k]));
+        if (v > amax) amax = v;
+      }
+      volatile float t = amax / 6.0f;
+      volatile float t2 = (gs > 0.0f) ? t / gs : 0.0f;
+      uint8_t sc = bsg_oracle_enc_e4m3(t2);
+      sf[m * KS + j] = sc;
+      volatile float denom = (float)bsg_oracle_dec_e4m3(sc) * gs;
+      uint8_t codes[16];
+      for (int64_t k = 0; k < 16; ++k) {
+        float v = bf16_bits_to_f32(x[j * 16 + k]);
+        volatile float q = (denom > 0.0f) ? v / denom : 0.0f;
+        codes[k] = bsg_oracle_enc_e2m1(q);
+      }
+      for (int64_t k = 0; k < 16; k += 2)
+        A[m * (K / 2) + (j * 16 + k) / 2] = (uint8_t)(codes[k] | (codes[k + 1] << 4));
+    }
+  }
+  return 0;
+}
+
 /* Threads the OpenMP loops above may use (for the timed CPU baseline). */
 int bsg_oracle_max_threads(void) {
 #ifdef _OPENMP
