@@ -107,6 +107,21 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 // Encodes a tiled descriptor after the same checks as the page's binding: extents >= box unless the
 // axis may run past the end, strides multiples of 16 bytes, 16-byte aligned base.
+struct DescKey {
+  const void* base;
+  int rank;
+  int swz;
+  uint64_t dims[5];
+  uint64_t strides[4];
+  uint32_t box[5];
+};
+struct DescCacheEntry {
+  DescKey key;
+  CUtensorMap map;
+  bool valid = false;
+};
+constexpr int kDescCacheSize = 8;
+
 bsg_status encode(CUtensorMap* map, const char* name, const void* base, int rank, const uint64_t* dims,
                   const uint64_t* strides_bytes, const uint32_t* box, const bool* allow_oob,
                   CUtensorMapSwizzle swz) {
@@ -126,6 +141,26 @@ bsg_status encode(CUtensorMap* map, const char* name, const void* base, int rank
       return fail(BSG_ERR_ALIGNMENT, "operand %s: stride %llu bytes (axis %d) must be a multiple of 16 below 2^40",
                   name, static_cast<unsigned long long>(strides_bytes[i]), i + 1);
   }
+  // A descriptor depends only on these arguments: repeated calls on the same buffers (the common case
+  // in a serving loop) reuse the last encodings of the calling thread instead of re-encoding.
+  DescKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = rank;
+  key.swz = static_cast<int>(swz);
+  for (int i = 0; i < rank; ++i) {
+    key.dims[i] = dims[i];
+    key.box[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) key.strides[i] = strides_bytes[i];
+  thread_local DescCacheEntry cache[kDescCacheSize];
+  thread_local int next_victim = 0;
+  for (int i = 0; i < kDescCacheSize; ++i) {
+    if (cache[i].valid && memcmp(&cache[i].key, &key, sizeof(key)) == 0) {
+      *map = cache[i].map;
+      return BSG_OK;
+    }
+  }
   cuuint64_t gdim[5], gstr[4];
   cuuint32_t bx[5], es[5];
   for (int i = 0; i < rank; ++i) {
@@ -138,6 +173,11 @@ bsg_status encode(CUtensorMap* map, const char* name, const void* base, int rank
                         gdim, gstr, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(BSG_ERR_CUDA, "cuTensorMapEncodeTiled of %s failed (CUresult %d)", name, (int)r);
+  DescCacheEntry& e = cache[next_victim];
+  next_victim = (next_victim + 1) % kDescCacheSize;
+  e.key = key;
+  e.map = *map;
+  e.valid = true;
   return BSG_OK;
 }
 
