@@ -100,9 +100,9 @@ def quant_fp8_rows(x: np.ndarray):
     xb = x.reshape(R, K // 128, 128)
     amax = np.abs(xb).max(axis=-1).astype(np.float32)
     scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
-    safe = np.where(scale > 0, scale, np.float32(1.0))
-    q = (xb / safe[..., None]).astype(np.float32)
-    q = np.where(scale[..., None] > 0, q, np.float32(0.0))
+    inv = np.where(scale > 0, np.float32(1.0) / np.where(scale > 0, scale, np.float32(1.0)),
+                   np.float32(0.0)).astype(np.float32)
+    q = (xb * inv[..., None]).astype(np.float32)
     return e4m3_encode(q).reshape(R, K), scale
 
 
@@ -117,9 +117,8 @@ def quant_fp8_blocks(w: np.ndarray):
         blk = w[nb * 128:(nb + 1) * 128].reshape(-1, K // 128, 128)
         amax = np.abs(blk).max(axis=(0, 2)).astype(np.float32)
         s = (amax / np.float32(E4M3_MAX)).astype(np.float32)
-        safe = np.where(s > 0, s, np.float32(1.0))
-        q = (blk / safe[None, :, None]).astype(np.float32)
-        q = np.where(s[None, :, None] > 0, q, np.float32(0.0))
+        inv = np.where(s > 0, np.float32(1.0) / np.where(s > 0, s, np.float32(1.0)), np.float32(0.0))
+        q = (blk * inv.astype(np.float32)[None, :, None]).astype(np.float32)
         codes[nb * 128:(nb + 1) * 128] = e4m3_encode(q).reshape(-1, K)
         scale[nb] = s
     return codes, scale
@@ -146,9 +145,9 @@ def quant_nvfp4(x: np.ndarray, gs: np.float32, chunk_rows: int = 4096):
             s_code = np.zeros(amax16.shape, dtype=np.uint8)
         s_val = e4m3_decode(s_code).astype(np.float32)
         denom = (s_val * gs).astype(np.float32)
-        safe = np.where(denom > 0, denom, np.float32(1.0))
-        q = (xb / safe[..., None]).astype(np.float32)
-        q = np.where(denom[..., None] > 0, q, np.float32(0.0))
+        inv = np.where(denom > 0, np.float32(1.0) / np.where(denom > 0, denom, np.float32(1.0)),
+                       np.float32(0.0)).astype(np.float32)
+        q = (xb * inv[..., None]).astype(np.float32)
         codes = e2m1_encode(q).reshape(-1, K)
         packed[r0:r0 + chunk_rows] = pack_e2m1(codes)
         sf[r0:r0 + chunk_rows] = s_code

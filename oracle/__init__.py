@@ -156,7 +156,7 @@ def enc_e2m1(x):
 
 def quant_fp8_rows(X_bf16_bits, M=None, src_rows=None, A=None, scale=None):
     """Activation quantisation to the FP8 GEMM's A operand: per 1 x 128 block, scale = amax/448,
-    code = e4m3_rne_satfinite(x / scale) in fp32.  X: uint16 bf16 bits [M_in, K]; output row m is
+    code = e4m3_rne_satfinite(x * (1 / scale)) in fp32 (one reciprocal per block).  X: uint16 bf16 bits [M_in, K]; output row m is
     input row src_rows[m] (or m).  Returns (A uint8 [M, K], scale f32 [M, K/128]); rows whose
     source is out of range keep the initial contents of A / scale (default 0xFF / NaN)."""
     L = lib()
@@ -176,8 +176,8 @@ def quant_fp8_rows(X_bf16_bits, M=None, src_rows=None, A=None, scale=None):
 
 def quant_nvfp4_rows(X_bf16_bits, gs, M=None, src_rows=None, A=None, sf=None):
     """Activation quantisation to the NVFP4 GEMM's A operand with global scale gs: per 1 x 16
-    block, s = ue4m3_rne_satfinite((amax/6)/gs), code = e2m1_rne_satfinite(x / (dec(s) * gs)), all in
-    fp32.  Returns (A uint8 [M, K/2] packed, low nibble = lower K; sf uint8 [M, K/16])."""
+    block, s = ue4m3_rne_satfinite((amax/6)/gs), code = e2m1_rne_satfinite(x * (1 / (dec(s) * gs))),
+    all in fp32.  Returns (A uint8 [M, K/2] packed, low nibble = lower K; sf uint8 [M, K/16])."""
     L = lib()
     X = np.ascontiguousarray(X_bf16_bits, dtype=np.uint16)
     M_in, K = X.shape

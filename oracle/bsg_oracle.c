@@ -205,14 +205,17 @@ int bsg_oracle_nvfp4(const uint8_t* A, const uint8_t* B, const uint8_t* sfa, con
  * contiguous runs; row m of the output is row src_rows[m] of the input).  Written from the format
  * definitions and the quantisation recipe of the two GEMMs' inputs:
  *
- *   FP8, per 1 x 128 block:  scale = amax / 448;  code = e4m3_rne_satfinite(x / scale)
+ *   FP8, per 1 x 128 block:  scale = amax / 448;  code = e4m3_rne_satfinite(x * (1 / scale))
  *   NVFP4, per 1 x 16 block, global scale gs:
- *       s = ue4m3_rne_satfinite((amax16 / 6) / gs);  code = e2m1_rne_satfinite(x / (dec(s) * gs))
+ *       s = ue4m3_rne_satfinite((amax16 / 6) / gs);  code = e2m1_rne_satfinite(x * (1 / (dec(s) * gs)))
  *
- * Every operation is the IEEE fp32 one (division and multiplication correctly rounded, no fused
- * multiply-add), because the quantised code is an integer decided in fp32 on the GPU as well.  A
- * block whose scale is zero gets all-zero codes.  The encoders round to the nearest representable
- * value, ties to the even code, and saturate at the largest finite magnitude (448, 6).
+ * Each element is multiplied by the reciprocal of its block's scale, computed once per block (the
+ * pages fix the scale, not how the division by it is carried out; one reciprocal per block and a
+ * product per element is how block quantisers are written).  Every operation is the IEEE fp32 one
+ * (division, reciprocal and product correctly rounded, no fused multiply-add), because the quantised
+ * code is an integer decided in fp32 on the GPU as well.  A block whose scale is zero gets all-zero
+ * codes.  The encoders round to the nearest representable value, ties to the even code, and
+ * saturate at the largest finite magnitude (448, 6).
  */
 
 /* fp32 -> E4M3 (FN) code: RNE, saturating at +-448; NaN -> 0x7F with the sign. */
@@ -279,9 +282,10 @@ int bsg_oracle_quant_fp8_rows(const uint16_t* X, const int32_t* src_rows, int64_
       }
       volatile float s = amax / 448.0f;
       scale[m * KB + kb] = s;
+      volatile float inv = (s > 0.0f) ? 1.0f / s : 0.0f;
       for (int64_t k = 0; k < 128; ++k) {
         float v = bf16_bits_to_f32(x[kb * 128 + k]);
-        volatile float q = (s > 0.0f) ? v / s : 0.0f;
+        volatile float q = v * inv;
         A[m * K + kb * 128 + k] = bsg_oracle_enc_e4m3(q);
       }
     }
@@ -311,10 +315,11 @@ int bsg_oracle_quant_nvfp4_rows(const uint16_t* X, const int32_t* src_rows, floa
       uint8_t sc = bsg_oracle_enc_e4m3(t2);
       sf[m * KS + j] = sc;
       volatile float denom = (float)bsg_oracle_dec_e4m3(sc) * gs;
+      volatile float inv = (denom > 0.0f) ? 1.0f / denom : 0.0f;
       uint8_t codes[16];
       for (int64_t k = 0; k < 16; ++k) {
         float v = bf16_bits_to_f32(x[j * 16 + k]);
-        volatile float q = (denom > 0.0f) ? v / denom : 0.0f;
+        volatile float q = v * inv;
         codes[k] = bsg_oracle_enc_e2m1(q);
       }
       for (int64_t k = 0; k < 16; k += 2)
