@@ -348,6 +348,49 @@ def roofline(w, per_launch_s, peaks, peak_src, sustained=False):
                            f"({w.kind} : bf16 nominal dense ratio)"}
 
 
+def time_quantiser(kind, M, K, peaks, steps=50, warmup=5):
+    """The step before the GEMM: BF16 activations [M, K], gathered through a random row permutation,
+    quantised into the GEMM's A operand.  HBM-bound; returns the also-line dict."""
+    import torch
+    import nvfp4_grouped_gemm_indices_b200 as bsg
+    g = torch.Generator(device="cuda").manual_seed(M + K)
+    X = torch.randn((M, K), device="cuda", generator=g).to(torch.bfloat16)
+    src = torch.randperm(M, device="cuda", generator=g).to(torch.int32)
+    if kind == "fp8":
+        A = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+        S = torch.empty((M, K // 128), dtype=torch.float32, device="cuda")
+        launch = lambda st: bsg.bsg_quantize_fp8_rows(X, src, A, S, M, M, K, st)
+        nbytes = 2 * M * K + M * K + 4 * M * (K // 128) + 4 * M
+    else:
+        gs = torch.tensor([float(X.float().abs().max()) / (448.0 * 6.0)], dtype=torch.float32, device="cuda")
+        A = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+        S = torch.empty((M, K // 16), dtype=torch.uint8, device="cuda")
+        launch = lambda st: bsg.bsg_quantize_nvfp4_rows(X, src, gs, A, S, M, M, K, st)
+        nbytes = 2 * M * K + M * K // 2 + M * (K // 16) + 4 * M
+    flush = make_flush() if 2 * M * K < 2 * L2_BYTES else None
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        launch(stream.cuda_stream)
+    torch.cuda.synchronize()
+    tot = 0.0
+    for _ in range(steps):
+        if flush is not None:
+            flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        launch(stream.cuda_stream)
+        b.record(stream)
+        b.synchronize()
+        tot += a.elapsed_time(b) / 1e3
+    per = tot / steps
+    ach = nbytes / per / 1e9
+    return {"us_per_launch": round(per * 1e6, 2),
+            "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None, "algorithmic_bytes": nbytes},
+            "l2": "flushed" if flush else "inputs > L2"}
+
+
 def cpu_baseline(w, seconds):
     """The oracle as it stands, on the host's cores, over a bounded sample of the workload's rows
     (all N columns each).  Returns (TFLOPS, cores, sample description)."""
@@ -458,6 +501,10 @@ def run_bsg(args):
                 also[wc.name] = {"tactic": r.tactic(), "tflops": round(wc.flops / pl / 1e12, 2),
                                  "us_per_launch": round(pl * 1e6, 2),
                                  "roofline": rf, "l2": "flushed" if fl else "inputs > L2"}
+            del r
+            torch.cuda.empty_cache()
+            also["quant_fp8_rows_gather_m8192_k7168"] = time_quantiser("fp8", 8192, 7168, peaks)
+            also["quant_nvfp4_rows_gather_m65536_k8192"] = time_quantiser("nvfp4", 65536, 8192, peaks)
             line["also"] = also
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -84,6 +84,35 @@ bsg_status bsg_nvfp4_gemm(const void* A, const void* B, const void* sfa, const v
                           const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G,
                           bsg_stream_t stream);
 
+/*
+ * Activation quantisation into the A operand of the GEMMs above (the step just before the GEMM), with
+ * an optional row gather -- the MoE "expand" that makes each expert's tokens contiguous, after the
+ * expand-and-quantise of the input rows in the ONNX Runtime page cited above, section 1.
+ *
+ *   for every output row m with r = (src_rows ? src_rows[m] : m) in [0, M_in):
+ *     FP8,   per 128-element block b:  a_scale[m,b] = amax / 448
+ *                                      A[m,k] = e4m3(X[r,k] * (1 / a_scale[m,b]))
+ *     NVFP4, per 16-element block j:   sfa[m,j]   = ue4m3((amax / 6) / gs)
+ *                                      A[m,k]     = e2m1(X[r,k] * (1 / (sfa[m,j] * gs)))
+ *   amax is the largest |X[r,k]| of the block; every step is an IEEE fp32 operation (the reciprocal
+ *   is taken once per block); e4m3 / e2m1 /
+ *   ue4m3 round to the nearest value, ties to the even code, and saturate at 448 / 6 / 448; a zero
+ *   block gets scale 0 and zero codes.  Output rows whose source is outside [0, M_in) are not written.
+ *
+ * X         bf16  [M_in, K]  activations (finite values), row-major, 16-byte aligned.
+ * src_rows  int32 [M]        source row of each output row, or NULL (then M <= M_in, row m <- row m).
+ * A         FP8: uint8 [M, K] (16-byte aligned); NVFP4: uint8 [M, K/2], two codes per byte, the lower-K
+ *           element in the low nibble (16-byte aligned) -- exactly the GEMMs' A layouts.
+ * a_scale   float [M, K/128] (4-byte aligned).   sfa  uint8 [M, K/16].
+ * global_scale  device float [1]: gs > 0 (for example amax(X) / (448 * 6)); read on the device.
+ * Contract: 1 <= M, M_in <= 2^31 - 1; FP8: K % 128 == 0; NVFP4: K % 16 == 0; 16 <= K <= 2^20.
+ * Asynchronous on `stream`; nothing is allocated or retained.
+ */
+bsg_status bsg_quantize_fp8_rows(const void* X, const int32_t* src_rows, void* A, float* a_scale, int64_t M_in,
+                                 int64_t M, int64_t K, bsg_stream_t stream);
+bsg_status bsg_quantize_nvfp4_rows(const void* X, const int32_t* src_rows, const float* global_scale, void* A,
+                                   void* sfa, int64_t M_in, int64_t M, int64_t K, bsg_stream_t stream);
+
 /* Description of the last failure on the calling thread ("" if none).  The string stays valid until
  * the next bsg_* call on the same thread. */
 const char* bsg_last_error(void);

@@ -14,6 +14,11 @@ Convenience wrappers infer the sizes from torch tensors and allocate C when not 
 
     fp8_grouped_gemm(A, B, a_scale, b_scale, m_indices, out=None)
     nvfp4_gemm(A, B, sfa, sfb, alpha, m_indices, out=None)
+
+and the step before the GEMM (activation quantisation with an optional row gather)::
+
+    quantize_fp8_rows(X, src_rows=None) -> (A, a_scale)
+    quantize_nvfp4_rows(X, global_scale, src_rows=None) -> (A, sfa)
 """
 from __future__ import annotations
 
@@ -41,6 +46,7 @@ EXPORTED = [
     "bsg_fp8_grouped_gemm", "bsg_nvfp4_gemm", "bsg_last_error", "bsg_get_device_status",
     "bsg_set_wait_timeout_ns", "bsg_num_tactics", "bsg_tactic_name", "bsg_choose_tactic",
     "bsg_tactic_score", "bsg_set_tactic", "bsg_set_max_ctas", "bsg_debug_set_fault", "bsg_version",
+    "bsg_quantize_fp8_rows", "bsg_quantize_nvfp4_rows",
 ]
 
 
@@ -89,6 +95,10 @@ def load(path: Optional[str] = None):
     L.bsg_debug_set_fault.argtypes = [i32]
     L.bsg_version.restype = ctypes.c_char_p
     L.bsg_version.argtypes = []
+    L.bsg_quantize_fp8_rows.restype = i32
+    L.bsg_quantize_fp8_rows.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
+    L.bsg_quantize_nvfp4_rows.restype = i32
+    L.bsg_quantize_nvfp4_rows.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
     if path is None:
         _lib = L
     return L
@@ -132,6 +142,16 @@ def bsg_fp8_grouped_gemm(A, B, a_scale, b_scale, m_indices, C, M, N, K, G, strea
 def bsg_nvfp4_gemm(A, B, sfa, sfb, alpha, m_indices, C, M, N, K, G, stream=None):
     _check(load().bsg_nvfp4_gemm(_ptr(A), _ptr(B), _ptr(sfa), _ptr(sfb), _ptr(alpha), _ptr(m_indices), _ptr(C),
                                  int(M), int(N), int(K), int(G), _stream(stream)))
+
+
+def bsg_quantize_fp8_rows(X, src_rows, A, a_scale, M_in, M, K, stream=None):
+    _check(load().bsg_quantize_fp8_rows(_ptr(X), _ptr(src_rows), _ptr(A), _ptr(a_scale), int(M_in), int(M), int(K),
+                                        _stream(stream)))
+
+
+def bsg_quantize_nvfp4_rows(X, src_rows, global_scale, A, sfa, M_in, M, K, stream=None):
+    _check(load().bsg_quantize_nvfp4_rows(_ptr(X), _ptr(src_rows), _ptr(global_scale), _ptr(A), _ptr(sfa),
+                                          int(M_in), int(M), int(K), _stream(stream)))
 
 
 def bsg_last_error() -> str:
@@ -259,3 +279,37 @@ def nvfp4_gemm(A, B, sfa, sfb, alpha, m_indices, out=None, stream=None):
         _need(out, torch.bfloat16, "out", 2)
     bsg_nvfp4_gemm(A, B, sfa, sfb, alpha, m_indices, out, M, N, K, G, stream)
     return out
+
+
+def quantize_fp8_rows(X, src_rows=None, stream=None):
+    """X bf16 [M_in, K] -> (A uint8 [M, K] E4M3 codes, a_scale f32 [M, K/128]), the FP8 GEMM's A
+    operand; with src_rows (int32 [M]) output row m is input row src_rows[m]."""
+    import torch
+    _need(X, torch.bfloat16, "X", 2)
+    M_in, K = X.shape
+    M = M_in
+    if src_rows is not None:
+        _need(src_rows, torch.int32, "src_rows", 1)
+        M = src_rows.numel()
+    A = torch.zeros((M, K), dtype=torch.uint8, device=X.device)
+    s = torch.zeros((M, K // 128), dtype=torch.float32, device=X.device)
+    bsg_quantize_fp8_rows(X, src_rows, A, s, M_in, M, K, stream)
+    return A, s
+
+
+def quantize_nvfp4_rows(X, global_scale, src_rows=None, stream=None):
+    """X bf16 [M_in, K], global_scale f32 [1] on the device -> (A uint8 [M, K/2] packed E2M1,
+    sfa uint8 [M, K/16]), the NVFP4 GEMM's A operand."""
+    import torch
+    _need(X, torch.bfloat16, "X", 2)
+    _need(global_scale, torch.float32, "global_scale")
+    M_in, K = X.shape
+    M = M_in
+    if src_rows is not None:
+        _need(src_rows, torch.int32, "src_rows", 1)
+        M = src_rows.numel()
+    A = torch.zeros((M, K // 2), dtype=torch.uint8, device=X.device)
+    sf = torch.zeros((M, K // 16), dtype=torch.uint8, device=X.device)
+    bsg_quantize_nvfp4_rows(X, src_rows, global_scale, A, sf, M_in, M, K, stream)
+    return A, sf
+

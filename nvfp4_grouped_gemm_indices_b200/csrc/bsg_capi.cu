@@ -18,6 +18,7 @@
 #include <string>
 
 #include "../../include/bsg.h"
+#include "bsg_quant.cuh"
 #include "bsg_chooser.h"
 #include "bsg_fp8.cuh"
 #include "bsg_nvfp4.cuh"
@@ -477,6 +478,80 @@ bsg_status bsg_nvfp4_gemm(const void* A, const void* B, const void* sfa, const v
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launch of the nvfp4 kernel");
+  return BSG_OK;
+}
+
+static bsg_status check_quant(const void* X, const int32_t* src_rows, const void* A, const void* scale, int64_t M_in,
+                              int64_t M, int64_t K, int64_t k_multiple) {
+  if (!X || !A || !scale) return fail(BSG_ERR_INVALID_ARG, "X, A and the scale output must be non-null");
+  if (M < 1 || M_in < 1 || M > 0x7FFFFFFFll || M_in > 0x7FFFFFFFll)
+    return fail(BSG_ERR_UNSUPPORTED_SHAPE, "M = %lld and M_in = %lld must lie in [1, 2^31 - 1]", (long long)M,
+                (long long)M_in);
+  if (!src_rows && M > M_in)
+    return fail(BSG_ERR_INVALID_ARG, "without src_rows every output row m reads input row m: M = %lld > M_in = %lld",
+                (long long)M, (long long)M_in);
+  if (K < 16 || K > (1ll << 20) || K % k_multiple != 0)
+    return fail(BSG_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a multiple of %lld in [16, 2^20]", (long long)K,
+                (long long)k_multiple);
+  if (!aligned(X, 16) || !aligned(A, 16)) return fail(BSG_ERR_ALIGNMENT, "X and A must be 16-byte aligned");
+  if (src_rows && !aligned(src_rows, 4)) return fail(BSG_ERR_ALIGNMENT, "src_rows must be 4-byte aligned");
+  return BSG_OK;
+}
+
+static int quant_grid(int sm_count, int64_t M, int64_t K, int64_t cols_per_task) {
+  const int64_t tasks = M * ((K + cols_per_task - 1) / cols_per_task);            // one warp each
+  const int64_t blocks = (tasks + bsg::quant::THREADS / 32 - 1) / (bsg::quant::THREADS / 32);
+  const int64_t cap = static_cast<int64_t>(sm_count) * (2048 / bsg::quant::THREADS);
+  return static_cast<int>(blocks < cap ? blocks : cap);
+}
+
+bsg_status bsg_quantize_fp8_rows(const void* X, const int32_t* src_rows, void* A, float* a_scale, int64_t M_in,
+                                 int64_t M, int64_t K, bsg_stream_t stream) {
+  g_last_error.clear();
+  bsg_status st = check_quant(X, src_rows, A, a_scale, M_in, M, K, 128);
+  if (st != BSG_OK) return st;
+  if (!aligned(a_scale, 4)) return fail(BSG_ERR_ALIGNMENT, "a_scale must be 4-byte aligned");
+  DeviceState* dev = nullptr;
+  if ((st = device_state(&dev)) != BSG_OK) return st;
+  bsg::quant::QuantParams p;
+  memset(&p, 0, sizeof(p));
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.src_rows = src_rows;
+  p.A = static_cast<uint8_t*>(A);
+  p.scale = a_scale;
+  p.M_in = M_in;
+  p.M = M;
+  p.K = static_cast<int>(K);
+  bsg::quant::bsg_quant_fp8_rows_kernel<<<quant_grid(dev->sm_count, M, K, bsg::quant::CHUNK * bsg::quant::GROUP), bsg::quant::THREADS, 0,
+                                          reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the fp8 quantisation kernel");
+  return BSG_OK;
+}
+
+bsg_status bsg_quantize_nvfp4_rows(const void* X, const int32_t* src_rows, const float* global_scale, void* A,
+                                   void* sfa, int64_t M_in, int64_t M, int64_t K, bsg_stream_t stream) {
+  g_last_error.clear();
+  bsg_status st = check_quant(X, src_rows, A, sfa, M_in, M, K, 16);
+  if (st != BSG_OK) return st;
+  if (!global_scale || !aligned(global_scale, 4))
+    return fail(BSG_ERR_INVALID_ARG, "global_scale must be a non-null, 4-byte aligned device pointer");
+  DeviceState* dev = nullptr;
+  if ((st = device_state(&dev)) != BSG_OK) return st;
+  bsg::quant::QuantParams p;
+  memset(&p, 0, sizeof(p));
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.src_rows = src_rows;
+  p.gs = global_scale;
+  p.A = static_cast<uint8_t*>(A);
+  p.scale = sfa;
+  p.M_in = M_in;
+  p.M = M;
+  p.K = static_cast<int>(K);
+  bsg::quant::bsg_quant_nvfp4_rows_kernel<<<quant_grid(dev->sm_count, M, K, bsg::quant::NV_CHUNK * bsg::quant::NV_GROUP), bsg::quant::THREADS, 0,
+                                            reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the nvfp4 quantisation kernel");
   return BSG_OK;
 }
 

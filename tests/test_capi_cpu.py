@@ -166,3 +166,28 @@ def test_set_max_ctas_validation(lib):
     with pytest.raises(bsg.BsgError):
         bsg.bsg_set_max_ctas(0, -1)
     bsg.bsg_set_max_ctas(0, 0)
+
+
+@pytest.mark.parametrize("fn,kw,status,needle", [
+    ("fp8", dict(X=0), bsg.BSG_ERR_INVALID_ARG, "non-null"),
+    ("fp8", dict(K=200), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "multiple of 128"),
+    ("fp8", dict(M=0), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "M = 0"),
+    ("fp8", dict(src_rows=0, M=20, M_in=10), bsg.BSG_ERR_INVALID_ARG, "M_in"),
+    ("fp8", dict(X=FAKE + 8), bsg.BSG_ERR_ALIGNMENT, "16-byte"),
+    ("fp8", dict(scale=FAKE + 2), bsg.BSG_ERR_ALIGNMENT, "a_scale"),
+    ("nvfp4", dict(K=24), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "multiple of 16"),
+    ("nvfp4", dict(gs=0), bsg.BSG_ERR_INVALID_ARG, "global_scale"),
+    ("nvfp4", dict(A=FAKE + 4), bsg.BSG_ERR_ALIGNMENT, "16-byte"),
+])
+def test_quantiser_argument_errors(lib, fn, kw, status, needle):
+    a = dict(X=FAKE, src_rows=FAKE, gs=FAKE, A=FAKE, scale=FAKE, M_in=64, M=64, K=256)
+    a.update(kw)
+    with pytest.raises(bsg.BsgError) as ei:
+        if fn == "fp8":
+            bsg.bsg_quantize_fp8_rows(a["X"], a["src_rows"] or None, a["A"], a["scale"], a["M_in"], a["M"], a["K"], stream=0)
+        else:
+            bsg.bsg_quantize_nvfp4_rows(a["X"], a["src_rows"] or None, a["gs"] or None, a["A"], a["scale"], a["M_in"],
+                                        a["M"], a["K"], stream=0)
+    assert ei.value.status == status
+    assert needle in str(ei.value)
+
