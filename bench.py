@@ -50,6 +50,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-also", action="store_true", help="skip the other workloads' kernel numbers")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--quant-only", action="store_true",
+                    help="time only the activation quantisers (one JSON line each) -- for profiling")
     return ap.parse_args(argv)
 
 
@@ -387,7 +389,9 @@ def time_quantiser(kind, M, K, peaks, steps=50, warmup=5):
     ach = nbytes / per / 1e9
     return {"us_per_launch": round(per * 1e6, 2),
             "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None, "algorithmic_bytes": nbytes},
+                         "frac": round(ach / peaks["hbm_gbs"], 4),
+                         "traffic": recorded_traffic(f"quant_{kind}_rows_gather_m{M}_k{K}"),
+                         "algorithmic_bytes": nbytes},
             "l2": "flushed" if flush else "inputs > L2"}
 
 
@@ -553,8 +557,20 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_quant_only(args):
+    import torch
+    torch.cuda.set_device(0)
+    peaks, _ = load_peaks()
+    for kind, M, K in (("fp8", 8192, 7168), ("nvfp4", 65536, 8192)):
+        d = time_quantiser(kind, M, K, peaks, steps=max(1, args.steps), warmup=max(1, args.warmup))
+        print(json.dumps({"kernel": f"quant_{kind}_rows_gather_m{M}_k{K}", **d}), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.quant_only:
+        run_quant_only(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:
