@@ -50,6 +50,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-also", action="store_true", help="skip the other workloads' kernel numbers")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every tactic on a set of shapes and compare with the chooser's pick")
     ap.add_argument("--quant-only", action="store_true",
                     help="time only the activation quantisers (one JSON line each) -- for profiling")
     return ap.parse_args(argv)
@@ -566,8 +568,57 @@ def run_quant_only(args):
         print(json.dumps({"kernel": f"quant_{kind}_rows_gather_m{M}_k{K}", **d}), flush=True)
 
 
+def sweep_shapes():
+    """The five workloads plus shapes that move the pick: few rows over many experts, a dense tail,
+    skewed and balanced routings."""
+    from nvfp4_grouped_gemm_indices_b200 import workloads as W
+    rng = np.random.default_rng(7)
+    out = [W.config(i) for i in range(5)]
+    for (M, N, K, G) in [(2048, 4096, 7168, 8), (4096, 2048, 4096, 16), (1024, 7168, 2048, 32), (16384, 4096, 4096, 4)]:
+        idx = W.counts_to_indices(rng.multinomial(M, [1.0 / G] * G))
+        out.append(W.make_fp8(M, N, K, G, idx, seed=M + N, name=f"fp8_sweep_g{G}_m{M}_n{N}_k{K}"))
+    for (M, N, K, G) in [(1024, 8192, 4096, 1), (8192, 4096, 4096, 8), (512, 16384, 8192, 4)]:
+        idx = W.counts_to_indices(rng.multinomial(M, [1.0 / G] * G))
+        out.append(W.make_nvfp4(M, N, K, G, idx, seed=M + N, name=f"nvfp4_sweep_g{G}_m{M}_n{N}_k{K}"))
+    return out
+
+
+def run_sweep(args):
+    """Every tactic on every sweep shape: prints one JSON line per shape with the time of each tactic,
+    the chooser's pick and its regret (time of the pick / best time)."""
+    import torch
+    import nvfp4_grouped_gemm_indices_b200 as bsg
+    torch.cuda.set_device(0)
+    sms = torch_sm_count()
+    regrets = []
+    for w in sweep_shapes():
+        kind = 0 if w.kind == "fp8" else 1
+        r = Runner(w)
+        flush = make_flush() if (w.A.nbytes + w.B.nbytes) < 2 * L2_BYTES else None
+        times = {}
+        for t in range(bsg.bsg_num_tactics(kind)):
+            bsg.bsg_set_tactic(kind, t)
+            _, per = time_kernel(r, max(10, min(args.steps, 100)), 3, flush)
+            times[bsg.bsg_tactic_name(kind, t)] = per
+        bsg.bsg_set_tactic(kind, -1)
+        pick = bsg.bsg_tactic_name(kind, bsg.bsg_choose_tactic(kind, w.M, w.N, w.K, w.G, sms))
+        best = min(times, key=times.get)
+        regret = times[pick] / times[best]
+        regrets.append(regret)
+        print(json.dumps({"shape": w.name, "us": {k: round(v * 1e6, 2) for k, v in times.items()},
+                          "chooser": pick, "best": best, "regret": round(regret, 4)}), flush=True)
+        del r
+        torch.cuda.empty_cache()
+    print(json.dumps({"shapes": len(regrets), "picks_best": sum(1 for x in regrets if x == 1.0),
+                      "geomean_regret": round(float(np.exp(np.mean(np.log(regrets)))), 4),
+                      "max_regret": round(max(regrets), 4)}), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.quant_only:
         run_quant_only(args)
         return
