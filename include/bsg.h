@@ -147,6 +147,24 @@ double bsg_tactic_score(int kind, int tactic, int64_t M, int64_t N, int64_t K, i
 bsg_status bsg_set_tactic(int kind, int tactic);
 
 /*
+ * Runtime tactic selection by measurement (the autotuning of the score-ranked candidates on the page
+ * "[flashinfer] FlashInfer의 FP4 GEMM 최적화: 휴리스틱 개선과 Autotuning 효율화", section 1; with two
+ * tactics per kind the top-N of the ranking is all of them): runs every tactic of the kind on the
+ * caller's operands -- one warm-up launch, then `reps` timed launches each,
+ * CUDA events on `stream` -- records the fastest for these exact sizes (M, N, K, G) in a per-process
+ * table that bsg_choose_tactic consults after a forced tactic and before the score, and returns its
+ * id (or a negative bsg_status).  The arguments are those of the GEMM call; C receives the correct
+ * result.  Synchronises `stream`; 1 <= reps <= 10000.  bsg_autotune_clear() empties the table.
+ */
+int bsg_autotune_fp8(const void* A, const void* B, const float* a_scale, const float* b_scale,
+                     const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G, int reps,
+                     bsg_stream_t stream);
+int bsg_autotune_nvfp4(const void* A, const void* B, const void* sfa, const void* sfb, const float* alpha,
+                       const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G, int reps,
+                       bsg_stream_t stream);
+void bsg_autotune_clear(void);
+
+/*
  * Upper bound on the persistent grid of later calls of one kind (0 = FP8, 1 = NVFP4); 0 restores the
  * default (one CTA per SM, fewer when there are fewer work units).  Any value >= 1 gives the same
  * results, only slower: each CTA then walks more work units through the same pipelines.

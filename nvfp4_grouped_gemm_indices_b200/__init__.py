@@ -46,7 +46,8 @@ EXPORTED = [
     "bsg_fp8_grouped_gemm", "bsg_nvfp4_gemm", "bsg_last_error", "bsg_get_device_status",
     "bsg_set_wait_timeout_ns", "bsg_num_tactics", "bsg_tactic_name", "bsg_choose_tactic",
     "bsg_tactic_score", "bsg_set_tactic", "bsg_set_max_ctas", "bsg_debug_set_fault", "bsg_version",
-    "bsg_quantize_fp8_rows", "bsg_quantize_nvfp4_rows",
+    "bsg_quantize_fp8_rows", "bsg_quantize_nvfp4_rows", "bsg_autotune_fp8", "bsg_autotune_nvfp4",
+    "bsg_autotune_clear",
 ]
 
 
@@ -97,6 +98,12 @@ def load(path: Optional[str] = None):
     L.bsg_version.argtypes = []
     L.bsg_quantize_fp8_rows.restype = i32
     L.bsg_quantize_fp8_rows.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
+    L.bsg_autotune_fp8.restype = i32
+    L.bsg_autotune_fp8.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, vp]
+    L.bsg_autotune_nvfp4.restype = i32
+    L.bsg_autotune_nvfp4.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, vp]
+    L.bsg_autotune_clear.restype = None
+    L.bsg_autotune_clear.argtypes = []
     L.bsg_quantize_nvfp4_rows.restype = i32
     L.bsg_quantize_nvfp4_rows.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
     if path is None:
@@ -152,6 +159,24 @@ def bsg_quantize_fp8_rows(X, src_rows, A, a_scale, M_in, M, K, stream=None):
 def bsg_quantize_nvfp4_rows(X, src_rows, global_scale, A, sfa, M_in, M, K, stream=None):
     _check(load().bsg_quantize_nvfp4_rows(_ptr(X), _ptr(src_rows), _ptr(global_scale), _ptr(A), _ptr(sfa),
                                           int(M_in), int(M), int(K), _stream(stream)))
+
+
+def bsg_autotune_fp8(A, B, a_scale, b_scale, m_indices, C, M, N, K, G, reps=20, stream=None) -> int:
+    r = int(load().bsg_autotune_fp8(_ptr(A), _ptr(B), _ptr(a_scale), _ptr(b_scale), _ptr(m_indices), _ptr(C),
+                                    int(M), int(N), int(K), int(G), int(reps), _stream(stream)))
+    _check(min(r, 0))
+    return r
+
+
+def bsg_autotune_nvfp4(A, B, sfa, sfb, alpha, m_indices, C, M, N, K, G, reps=20, stream=None) -> int:
+    r = int(load().bsg_autotune_nvfp4(_ptr(A), _ptr(B), _ptr(sfa), _ptr(sfb), _ptr(alpha), _ptr(m_indices),
+                                      _ptr(C), int(M), int(N), int(K), int(G), int(reps), _stream(stream)))
+    _check(min(r, 0))
+    return r
+
+
+def bsg_autotune_clear():
+    load().bsg_autotune_clear()
 
 
 def bsg_last_error() -> str:

@@ -253,10 +253,13 @@ bsg_status bsg_debug_set_fault(int mode) {
   return BSG_OK;
 }
 
-bsg_status bsg_fp8_grouped_gemm(const void* A, const void* B, const float* a_scale, const float* b_scale,
-                                const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G,
-                                bsg_stream_t stream) {
-  g_last_error.clear();
+}  // extern "C"
+
+namespace {
+
+bsg_status fp8_check(const void* A, const void* B, const float* a_scale, const float* b_scale,
+                     const int32_t* m_indices, const void* C, int64_t M, int64_t N, int64_t K, int64_t G,
+                     DeviceState** dev_out) {
   bsg_status st = check_common(A, B, m_indices, C, M, N, K, G);
   if (st != BSG_OK) return st;
   if (!a_scale || !b_scale) return fail(BSG_ERR_INVALID_ARG, "a_scale and b_scale must be non-null");
@@ -266,11 +269,14 @@ bsg_status bsg_fp8_grouped_gemm(const void* A, const void* B, const float* a_sca
   if (!aligned(A, 16) || !aligned(B, 16)) return fail(BSG_ERR_ALIGNMENT, "A and B must be 16-byte aligned");
   if (!aligned(a_scale, 4) || !aligned(b_scale, 4))
     return fail(BSG_ERR_ALIGNMENT, "a_scale and b_scale must be 4-byte aligned");
-  DeviceState* dev = nullptr;
-  if ((st = device_state(&dev)) != BSG_OK) return st;
+  return device_state(dev_out);
+}
 
-  // tactic 0: one SM per 128 x 256 tile; tactic 1: an SM pair per 256 x 256 tile (cta_group::2)
-  const int tactic = bsg_choose_tactic(0, M, N, K, G, dev->sm_count);
+// tactic 0: one SM per 128 x 256 tile; tactic 1: an SM pair per 256 x 256 tile (cta_group::2)
+bsg_status fp8_launch(DeviceState* dev, const void* A, const void* B, const float* a_scale, const float* b_scale,
+                      const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G,
+                      bsg_stream_t stream, int tactic) {
+  bsg_status st;
   const int cg = tactic == 1 ? 2 : 1;
 
   bsg::Fp8Params p;
@@ -361,10 +367,9 @@ bsg_status bsg_fp8_grouped_gemm(const void* A, const void* B, const float* a_sca
   return BSG_OK;
 }
 
-bsg_status bsg_nvfp4_gemm(const void* A, const void* B, const void* sfa, const void* sfb, const float* alpha,
-                          const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G,
-                          bsg_stream_t stream) {
-  g_last_error.clear();
+bsg_status nvfp4_check(const void* A, const void* B, const void* sfa, const void* sfb, const float* alpha,
+                       const int32_t* m_indices, const void* C, int64_t M, int64_t N, int64_t K, int64_t G,
+                       DeviceState** dev_out) {
   bsg_status st = check_common(A, B, m_indices, C, M, N, K, G);
   if (st != BSG_OK) return st;
   if (!sfa || !sfb || !alpha) return fail(BSG_ERR_INVALID_ARG, "sfa, sfb and alpha must be non-null");
@@ -373,11 +378,14 @@ bsg_status bsg_nvfp4_gemm(const void* A, const void* B, const void* sfa, const v
                 "K = %lld must be a positive multiple of 256 (16-byte rows of packed codes and of scale bytes)",
                 (long long)K);
   if (!aligned(alpha, 4)) return fail(BSG_ERR_ALIGNMENT, "alpha must be 4-byte aligned");
-  DeviceState* dev = nullptr;
-  if ((st = device_state(&dev)) != BSG_OK) return st;
+  return device_state(dev_out);
+}
 
-  // tactic 0: one SM per 128 x 256 tile; tactic 1: an SM pair per 256 x 256 tile (cta_group::2)
-  const int tactic = bsg_choose_tactic(1, M, N, K, G, dev->sm_count);
+// tactic 0: one SM per 128 x 256 tile; tactic 1: an SM pair per 256 x 256 tile (cta_group::2)
+bsg_status nvfp4_launch(DeviceState* dev, const void* A, const void* B, const void* sfa, const void* sfb,
+                        const float* alpha, const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K,
+                        int64_t G, bsg_stream_t stream, int tactic) {
+  bsg_status st;
   const int cg = tactic == 1 ? 2 : 1;
 
   bsg::Nvfp4Params p;
@@ -479,6 +487,100 @@ bsg_status bsg_nvfp4_gemm(const void* A, const void* B, const void* sfa, const v
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launch of the nvfp4 kernel");
   return BSG_OK;
+}
+
+// Times `reps` launches of every tactic (after one warm-up launch each) with CUDA events on the
+// stream; returns the fastest tactic or a negative status.  `launch(t)` enqueues one call.
+template <typename Launch>
+int time_tactics(int kind, int reps, bsg_stream_t stream, Launch launch) {
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cudaEvent_t ev[2];
+  if (cudaEventCreate(&ev[0]) != cudaSuccess) return cuda_fail(cudaGetLastError(), "cudaEventCreate");
+  if (cudaEventCreate(&ev[1]) != cudaSuccess) {
+    cudaEventDestroy(ev[0]);
+    return cuda_fail(cudaGetLastError(), "cudaEventCreate");
+  }
+  int best = BSG_ERR_CUDA;
+  float best_ms = 0.f;
+  const int n = bsg_num_tactics(kind);
+  bsg_status st = BSG_OK;
+  for (int t = 0; t < n && st == BSG_OK; ++t) {
+    if ((st = launch(t)) != BSG_OK) break;
+    cudaEventRecord(ev[0], cs);
+    for (int r = 0; r < reps && st == BSG_OK; ++r) st = launch(t);
+    cudaEventRecord(ev[1], cs);
+    cudaError_t e = cudaEventSynchronize(ev[1]);
+    if (st != BSG_OK) break;
+    if (e != cudaSuccess) {
+      st = cuda_fail(e, "timing a tactic");
+      break;
+    }
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, ev[0], ev[1]);
+    if (best < 0 || ms < best_ms) {
+      best = t;
+      best_ms = ms;
+    }
+  }
+  cudaEventDestroy(ev[0]);
+  cudaEventDestroy(ev[1]);
+  return st != BSG_OK ? static_cast<int>(st) : best;
+}
+
+}  // namespace
+
+extern "C" {
+
+bsg_status bsg_fp8_grouped_gemm(const void* A, const void* B, const float* a_scale, const float* b_scale,
+                                const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G,
+                                bsg_stream_t stream) {
+  g_last_error.clear();
+  DeviceState* dev = nullptr;
+  bsg_status st = fp8_check(A, B, a_scale, b_scale, m_indices, C, M, N, K, G, &dev);
+  if (st != BSG_OK) return st;
+  const int tactic = bsg_choose_tactic(0, M, N, K, G, dev->sm_count);
+  return fp8_launch(dev, A, B, a_scale, b_scale, m_indices, C, M, N, K, G, stream, tactic);
+}
+
+bsg_status bsg_nvfp4_gemm(const void* A, const void* B, const void* sfa, const void* sfb, const float* alpha,
+                          const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G,
+                          bsg_stream_t stream) {
+  g_last_error.clear();
+  DeviceState* dev = nullptr;
+  bsg_status st = nvfp4_check(A, B, sfa, sfb, alpha, m_indices, C, M, N, K, G, &dev);
+  if (st != BSG_OK) return st;
+  const int tactic = bsg_choose_tactic(1, M, N, K, G, dev->sm_count);
+  return nvfp4_launch(dev, A, B, sfa, sfb, alpha, m_indices, C, M, N, K, G, stream, tactic);
+}
+
+int bsg_autotune_fp8(const void* A, const void* B, const float* a_scale, const float* b_scale,
+                     const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G, int reps,
+                     bsg_stream_t stream) {
+  g_last_error.clear();
+  if (reps < 1 || reps > 10000) return fail(BSG_ERR_INVALID_ARG, "reps = %d outside [1, 10000]", reps);
+  DeviceState* dev = nullptr;
+  bsg_status st = fp8_check(A, B, a_scale, b_scale, m_indices, C, M, N, K, G, &dev);
+  if (st != BSG_OK) return st;
+  const int best = time_tactics(0, reps, stream, [&](int t) {
+    return fp8_launch(dev, A, B, a_scale, b_scale, m_indices, C, M, N, K, G, stream, t);
+  });
+  if (best >= 0) bsg_record_tuned(0, M, N, K, G, best);
+  return best;
+}
+
+int bsg_autotune_nvfp4(const void* A, const void* B, const void* sfa, const void* sfb, const float* alpha,
+                       const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G, int reps,
+                       bsg_stream_t stream) {
+  g_last_error.clear();
+  if (reps < 1 || reps > 10000) return fail(BSG_ERR_INVALID_ARG, "reps = %d outside [1, 10000]", reps);
+  DeviceState* dev = nullptr;
+  bsg_status st = nvfp4_check(A, B, sfa, sfb, alpha, m_indices, C, M, N, K, G, &dev);
+  if (st != BSG_OK) return st;
+  const int best = time_tactics(1, reps, stream, [&](int t) {
+    return nvfp4_launch(dev, A, B, sfa, sfb, alpha, m_indices, C, M, N, K, G, stream, t);
+  });
+  if (best >= 0) bsg_record_tuned(1, M, N, K, G, best);
+  return best;
 }
 
 static bsg_status check_quant(const void* X, const int32_t* src_rows, const void* A, const void* scale, int64_t M_in,

@@ -18,7 +18,9 @@
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "../../include/bsg.h"
 #include "bsg_chooser.h"
@@ -59,6 +61,7 @@ const Tactic* table(int kind, int* n) {
 
 std::mutex g_mu;
 int g_forced_tactic[2] = {-1, -1};
+std::map<std::tuple<int, int64_t, int64_t, int64_t, int64_t>, int> g_tuned;
 int g_max_ctas[2] = {0, 0};
 bool g_env_read = false;
 
@@ -80,6 +83,17 @@ BsgUnitEstimate bsg_estimate_units(int64_t M, int64_t G) {
   e.segments = e.windows + runs - 1;
   e.pairs = (e.segments + 1) / 2 + runs / 2;
   return e;
+}
+
+void bsg_record_tuned(int kind, int64_t M, int64_t N, int64_t K, int64_t G, int tactic) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_tuned[std::make_tuple(kind, M, N, K, G)] = tactic;
+}
+
+int bsg_tuned_tactic(int kind, int64_t M, int64_t N, int64_t K, int64_t G) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto it = g_tuned.find(std::make_tuple(kind, M, N, K, G));
+  return it == g_tuned.end() ? -1 : it->second;
 }
 
 int bsg_forced_grid(int kind, int grid) {
@@ -136,6 +150,8 @@ int bsg_choose_tactic(int kind, int64_t M, int64_t N, int64_t K, int64_t G, int 
     read_env();
     int f = g_forced_tactic[kind];
     if (f >= 0 && f < n) return f;
+    auto it = g_tuned.find(std::make_tuple(kind, M, N, K, G));
+    if (it != g_tuned.end() && it->second >= 0 && it->second < n) return it->second;
   }
   int best = 0;
   double best_score = -1.0;
@@ -157,6 +173,11 @@ bsg_status bsg_set_tactic(int kind, int tactic) {
   read_env();
   g_forced_tactic[kind] = tactic < 0 ? -1 : tactic;
   return BSG_OK;
+}
+
+void bsg_autotune_clear(void) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_tuned.clear();
 }
 
 bsg_status bsg_set_max_ctas(int kind, int max_ctas) {

@@ -12,3 +12,9 @@ struct BsgUnitEstimate {
   int64_t pairs;      // pairs of same-expert segments (2-SM tiles)
 };
 BsgUnitEstimate bsg_estimate_units(int64_t M, int64_t G);
+
+// Measured winners (bsg_autotune_*) for exact problem sizes; bsg_choose_tactic prefers them to the
+// score.  bsg_tuned_tactic returns -1 when the sizes were never tuned.
+void bsg_record_tuned(int kind, int64_t M, int64_t N, int64_t K, int64_t G, int tactic);
+int bsg_tuned_tactic(int kind, int64_t M, int64_t N, int64_t K, int64_t G);
+

@@ -191,3 +191,13 @@ def test_quantiser_argument_errors(lib, fn, kw, status, needle):
     assert ei.value.status == status
     assert needle in str(ei.value)
 
+
+def test_autotune_argument_errors(lib):
+    with pytest.raises(bsg.BsgError) as ei:
+        bsg.bsg_autotune_fp8(**fp8_args(), reps=0, stream=0)
+    assert ei.value.status == bsg.BSG_ERR_INVALID_ARG and "reps" in str(ei.value)
+    with pytest.raises(bsg.BsgError) as ei:
+        bsg.bsg_autotune_nvfp4(**nvfp4_args(K=128), reps=5, stream=0)
+    assert ei.value.status == bsg.BSG_ERR_UNSUPPORTED_SHAPE
+    bsg.bsg_autotune_clear()
+

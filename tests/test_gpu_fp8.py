@@ -225,3 +225,21 @@ def test_fp8_torch_wrapper():
     out = bits(C)
     out[~routed] = SENTINEL  # the wrapper's fresh C is zero-filled
     compare(out, ref, routed)
+
+
+def test_fp8_autotune_records_the_measured_winner_and_stays_correct():
+    """Runtime autotune: every tactic runs on the caller's operands, the fastest is recorded for these
+    sizes and picked by the chooser afterwards; C holds the correct result."""
+    w = W.make_fp8(1024, 1024, 1024, 4, W.counts_to_indices([256, 300, 200, 268]), seed=44)
+    d = DevWorkload(w)
+    C = sentinel_out(w.M, w.N)
+    bsg.bsg_autotune_clear()
+    try:
+        t = bsg.bsg_autotune_fp8(d.A, d.B, d.a_scale, d.b_scale, d.m_indices, C, w.M, w.N, w.K, w.G, reps=5)
+        torch.cuda.synchronize()
+        assert 0 <= t < bsg.bsg_num_tactics(0)
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        assert bsg.bsg_choose_tactic(0, w.M, w.N, w.K, w.G, sms) == t
+        compare(bits(C), oracle_rows(w), routed_mask(w))
+    finally:
+        bsg.bsg_autotune_clear()

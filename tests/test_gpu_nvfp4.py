@@ -179,3 +179,21 @@ def test_nvfp4_bounded_wait_reports_timeout_and_context_survives():
         bsg.bsg_debug_set_fault(0)
         bsg.bsg_set_wait_timeout_ns(prev)
     full_check(w)
+
+
+def test_nvfp4_autotune_records_the_measured_winner_and_stays_correct():
+    rng = np.random.default_rng(45)
+    w = W.make_nvfp4(512, 1024, 1024, 2, W.counts_to_indices(rng.multinomial(512, [0.5, 0.5])), seed=45)
+    d = DevWorkload(w)
+    C = sentinel_out(w.M, w.N)
+    bsg.bsg_autotune_clear()
+    try:
+        bsg.bsg_set_tactic(1, -1)
+        t = bsg.bsg_autotune_nvfp4(d.A, d.B, d.sfa, d.sfb, d.alpha, d.m_indices, C, w.M, w.N, w.K, w.G, reps=5)
+        torch.cuda.synchronize()
+        assert 0 <= t < bsg.bsg_num_tactics(1)
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        assert bsg.bsg_choose_tactic(1, w.M, w.N, w.K, w.G, sms) == t
+        compare(bits(C), oracle_rows(w), routed_mask(w))
+    finally:
+        bsg.bsg_autotune_clear()
