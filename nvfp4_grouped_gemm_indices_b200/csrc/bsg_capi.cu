@@ -344,7 +344,7 @@ bsg_status fp8_launch(DeviceState* dev, const void* A, const void* B, const floa
     if (dev->fp8_pair_clusters < 1) return fail(BSG_ERR_CUDA, "no SM-pair cluster fits on this device");
     const BsgUnitEstimate est = bsg_estimate_units(M, G);
     const int64_t n_tiles = (N + bn - 1) / bn;
-    int64_t clusters = est.pairs * n_tiles;
+    int64_t clusters = est.pairs_max * n_tiles;
     if (clusters > dev->fp8_pair_clusters) clusters = dev->fp8_pair_clusters;
     const int grid = 2 * ((bsg_forced_grid(0, static_cast<int>(2 * clusters)) + 1) / 2);
     cudaLaunchConfig_t lc = {};
@@ -466,7 +466,7 @@ bsg_status nvfp4_launch(DeviceState* dev, const void* A, const void* B, const vo
     if (dev->nvfp4_pair_clusters < 1) return fail(BSG_ERR_CUDA, "no SM-pair cluster fits on this device");
     const BsgUnitEstimate est = bsg_estimate_units(M, G);
     const int64_t n_tiles = (N + bsg::nvfp4::BN - 1) / bsg::nvfp4::BN;
-    int64_t clusters = est.pairs * n_tiles;
+    int64_t clusters = est.pairs_max * n_tiles;
     if (clusters > dev->nvfp4_pair_clusters) clusters = dev->nvfp4_pair_clusters;
     const int grid = 2 * ((bsg_forced_grid(1, static_cast<int>(2 * clusters)) + 1) / 2);
     cudaLaunchConfig_t lc = {};

@@ -81,7 +81,13 @@ BsgUnitEstimate bsg_estimate_units(int64_t M, int64_t G) {
   e.windows = (M + 127) / 128;
   const int64_t runs = G < M ? G : M;
   e.segments = e.windows + runs - 1;
-  e.pairs = (e.segments + 1) / 2 + runs / 2;
+  // pairs: the scheduler pairs consecutive segments of one run, so a run cut into s segments gives
+  // ceil(s / 2) pairs; with R equal runs each spans ceil(M / (128 R)) windows, plus one more when
+  // runs start at arbitrary rows (R > 1)
+  const int64_t span = (M + 128 * runs - 1) / (128 * runs) + (runs > 1 ? 1 : 0);
+  e.pairs_max = (e.segments + 1) / 2 + runs / 2;
+  e.pairs = runs * ((span + 1) / 2);
+  if (e.pairs > e.pairs_max) e.pairs = e.pairs_max;
   return e;
 }
 

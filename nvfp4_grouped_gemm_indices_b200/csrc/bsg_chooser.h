@@ -9,7 +9,8 @@ int bsg_forced_grid(int kind, int grid);
 struct BsgUnitEstimate {
   int64_t windows;    // ceil(M / 128)
   int64_t segments;   // window segments: windows + (runs - 1), runs <= min(G, M)
-  int64_t pairs;      // pairs of same-expert segments (2-SM tiles)
+  int64_t pairs;      // expected pairs of same-expert segments (2-SM tiles): runs * ceil(span / 2)
+  int64_t pairs_max;  // upper bound on the pairs the scheduler can form (sizes the SM-pair grid)
 };
 BsgUnitEstimate bsg_estimate_units(int64_t M, int64_t G);
 

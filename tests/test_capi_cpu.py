@@ -133,7 +133,8 @@ def test_chooser_score_follows_the_page_formula(lib):
     # FP8 one-SM tactic 0 on M=8192 (64 windows), G=8: 71 segments, N=4096 -> 16 tiles of 256
     thr = {"fp8_1sm_m128_n256_s4": 0.47, "fp8_2sm_m256_n256_s6": 0.45}
     assert bsg.bsg_tactic_name(0, 0) in thr
-    segs, pairs = 64 + 8 - 1, (64 + 8 - 1 + 1) // 2 + 8 // 2
+    # 8 runs of 1024 rows: each spans 8 windows + 1 (arbitrary start) = 9 segments -> 5 pairs
+    segs, pairs = 64 + 8 - 1, 8 * 5
     t0 = bsg.bsg_tactic_name(0, 0)
     s = bsg.bsg_tactic_score(0, 0, 8192, 4096, 7168, 8, 148)
     waves = -(-(segs * 16) // 148)
