@@ -243,3 +243,42 @@ def test_fp8_autotune_records_the_measured_winner_and_stays_correct():
         compare(bits(C), oracle_rows(w), routed_mask(w))
     finally:
         bsg.bsg_autotune_clear()
+
+
+def test_fp8_no_routed_rows_writes_nothing(tactic):
+    """Every index out of range: the kernel hands out no unit and C stays untouched."""
+    M, N, K, G = 300, 256, 256, 3
+    idx = np.full(M, -1, np.int32)
+    idx[::7] = G + 5
+    w = W.make_fp8(M, N, K, G, idx, seed=9)
+    out = bits(DevWorkload(w).run())
+    bsg.bsg_get_device_status()
+    assert np.all(out == SENTINEL)
+
+
+def test_fp8_max_rows_and_max_experts():
+    """The launch contract's extremes: M = 2^24 rows (two experts, a run boundary off the window
+    grid) checked on sampled rows, and G = 4096 experts with one row each for a few of them."""
+    M, N, K, G = 1 << 24, 64, 128, 2
+    rng = np.random.default_rng(77)
+    A = rng.integers(0, 0x7E, (M, K), dtype=np.uint8)          # finite E4M3 codes
+    B = rng.integers(0, 0x7E, (G, N, K), dtype=np.uint8)
+    a_scale = rng.uniform(0.5, 2.0, (M, 1)).astype(np.float32)
+    b_scale = rng.uniform(0.5, 2.0, (G, 1, 1)).astype(np.float32)
+    idx = np.zeros(M, np.int32)
+    idx[(M // 2) + 37:] = 1
+    w = W.Workload("fp8_max_m", "fp8", M, N, K, G, A, B, idx, a_scale=a_scale, b_scale=b_scale)
+    d = DevWorkload(w)
+    out = bits(d.run())
+    bsg.bsg_get_device_status()
+    rows = np.unique(np.concatenate([np.arange(0, 64), np.arange(M // 2, M // 2 + 128), np.arange(M - 64, M),
+                                     rng.integers(0, M, 256)]))
+    compare(out[rows], oracle_rows(w, rows), routed_mask(w, rows))
+    del d
+    torch.cuda.empty_cache()
+    G2, M2 = 4096, 600
+    idx2 = np.full(M2, -1, np.int32)
+    idx2[rng.choice(M2, 40, replace=False)] = rng.choice(G2, 40, replace=False).astype(np.int32)
+    idx2 = np.sort(idx2)
+    w2 = W.make_fp8(M2, 64, 128, G2, idx2, seed=78)
+    compare(bits(DevWorkload(w2).run()), oracle_rows(w2), routed_mask(w2))
