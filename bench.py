@@ -577,6 +577,12 @@ def sweep_shapes():
     for (M, N, K, G) in [(2048, 4096, 7168, 8), (4096, 2048, 4096, 16), (1024, 7168, 2048, 32), (16384, 4096, 4096, 4)]:
         idx = W.counts_to_indices(rng.multinomial(M, [1.0 / G] * G))
         out.append(W.make_fp8(M, N, K, G, idx, seed=M + N, name=f"fp8_sweep_g{G}_m{M}_n{N}_k{K}"))
+    # few rows per expert (decode): where the operand-swapped tiles take over from the row tiles
+    idx = W.routing_zipf(96, 32, rng)
+    out.append(W.make_fp8(96, 2048, 4096, 32, idx, seed=96, name="fp8_sweep_zipf_g32_m96_n2048_k4096"))
+    for (M, N, K, G) in [(256, 4096, 2048, 16), (512, 4096, 4096, 8), (1024, 4096, 4096, 8)]:
+        idx = W.counts_to_indices(rng.multinomial(M, [1.0 / G] * G))
+        out.append(W.make_fp8(M, N, K, G, idx, seed=M + N + G, name=f"fp8_sweep_g{G}_m{M}_n{N}_k{K}"))
     for (M, N, K, G) in [(1024, 8192, 4096, 1), (8192, 4096, 4096, 8), (512, 16384, 8192, 4)]:
         idx = W.counts_to_indices(rng.multinomial(M, [1.0 / G] * G))
         out.append(W.make_nvfp4(M, N, K, G, idx, seed=M + N, name=f"nvfp4_sweep_g{G}_m{M}_n{N}_k{K}"))

@@ -139,6 +139,12 @@ uint64_t bsg_set_wait_timeout_ns(uint64_t ns);
  * from the sizes alone; bsg_choose_tactic() returns the best-scored (or forced) tactic, or a
  * negative bsg_status.  bsg_set_tactic() forces a tactic for later calls of that kind (-1 = let the
  * chooser decide); the environment variable BSG_TACTIC does the same at load time.
+ * FP8 tactics: 0 = one SM per 128-row window segment x 256 columns; 1 = an SM pair per 256 x 256
+ * tile; 2, 3 = operand-swapped tiles for experts with few rows (128 or 256 output columns x a chunk
+ * of at most 128 or 64 of one expert's rows; the page "[onnxruntime] ONNX Runtime: Blackwell
+ * (SM120+)에서 NVFP4 QMoE를 위한 네이티브 FP4xFP4 Prefill 최적화", section 1, keeps decode shapes on a
+ * path of their own).  NVFP4 tactics: 0 = one SM, 1 = an SM pair.  Every tactic computes the same
+ * result within the stated tolerance.
  */
 int bsg_num_tactics(int kind);
 const char* bsg_tactic_name(int kind, int tactic);
@@ -148,8 +154,8 @@ bsg_status bsg_set_tactic(int kind, int tactic);
 
 /*
  * Runtime tactic selection by measurement (the autotuning of the score-ranked candidates on the page
- * "[flashinfer] FlashInfer의 FP4 GEMM 최적화: 휴리스틱 개선과 Autotuning 효율화", section 1; with two
- * tactics per kind the top-N of the ranking is all of them): runs every tactic of the kind on the
+ * "[flashinfer] FlashInfer의 FP4 GEMM 최적화: 휴리스틱 개선과 Autotuning 효율화", section 1; with at most
+ * four tactics per kind the top-N of the ranking is all of them): runs every tactic of the kind on the
  * caller's operands -- one warm-up launch, then `reps` timed launches each,
  * CUDA events on `stream` -- records the fastest for these exact sizes (M, N, K, G) in a per-process
  * table that bsg_choose_tactic consults after a forced tactic and before the score, and returns its

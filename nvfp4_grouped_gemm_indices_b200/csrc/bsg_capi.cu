@@ -21,6 +21,7 @@
 #include "bsg_quant.cuh"
 #include "bsg_chooser.h"
 #include "bsg_fp8.cuh"
+#include "bsg_fp8_swap.cuh"
 #include "bsg_nvfp4.cuh"
 
 #define BSG_VERSION_STRING "bsg 0.1.0 (sm_100a)"
@@ -51,6 +52,7 @@ struct DeviceState {
   int sm_count = 0;
   bsg::DeviceStatus* status = nullptr;
   bool fp8_attr = false;
+  bool fp8_swap_attr = false;
   bool nvfp4_attr = false;
   int fp8_pair_clusters = 0;
   int nvfp4_pair_clusters = 0;
@@ -272,10 +274,79 @@ bsg_status fp8_check(const void* A, const void* B, const float* a_scale, const f
   return device_state(dev_out);
 }
 
-// tactic 0: one SM per 128 x 256 tile; tactic 1: an SM pair per 256 x 256 tile (cta_group::2)
+// tactics 2 and 3: the operand-swapped kernel for experts with few rows; 128 (tactic 2) or 256
+// (tactic 3) output columns per unit, token chunks of at most 128 / 64 rows
+bsg_status fp8_swap_launch(DeviceState* dev, const void* A, const void* B, const float* a_scale,
+                           const float* b_scale, const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K,
+                           int64_t G, bsg_stream_t stream, int tactic) {
+  bsg_status st;
+  const int nh = tactic == 3 ? 2 : 1;
+  const int bnr = 128 * nh;
+  bsg::Fp8Params p;
+  memset(&p, 0, sizeof(p));
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+    const uint64_t str[1] = {static_cast<uint64_t>(K)};
+    const uint32_t box[2] = {128u, static_cast<uint32_t>(bsg::fp8s::A_BOX)};
+    const bool oob[2] = {false, true};  // a chunk's last box may run past M: zero-filled, never stored
+    if ((st = encode(&p.tmA, "A", A, 2, dims, str, box, oob, CU_TENSOR_MAP_SWIZZLE_128B)) != BSG_OK) return st;
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), static_cast<uint64_t>(G)};
+    const uint64_t str[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N) * static_cast<uint64_t>(K)};
+    const uint32_t box[3] = {128u, static_cast<uint32_t>(bnr), 1u};
+    const bool oob[3] = {false, true, false};
+    if ((st = encode(&p.tmB, "B", B, 3, dims, str, box, oob, CU_TENSOR_MAP_SWIZZLE_128B)) != BSG_OK) return st;
+  }
+  p.a_scale = a_scale;
+  p.b_scale = b_scale;
+  p.m_indices = m_indices;
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.G = static_cast<int>(G);
+  // few windows: N tile outermost, so consecutive chunks of one expert (a run crossing a window
+  // boundary) read the same B tile at the same time; otherwise the usual raster groups
+  const int64_t windows = (M + 127) / 128;
+  p.n_group = windows <= 32 ? 1 : n_group_for(N, K, bnr);
+  p.timeout_ns = current_timeout();
+  p.status = dev->status;
+  p.debug_mode = current_fault();
+
+  cudaError_t e;
+  if (!dev->fp8_swap_attr) {
+    e = cudaFuncSetAttribute(bsg::fp8s::bsg_fp8_swap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bsg::fp8s::smem_bytes<1>()));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fp8 swapped kernel smem)");
+    e = cudaFuncSetAttribute(bsg::fp8s::bsg_fp8_swap_n256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bsg::fp8s::smem_bytes<2>()));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fp8 swapped 256-column kernel smem)");
+    dev->fp8_swap_attr = true;
+  }
+  // units: chunks x N tiles; sorted routing gives at most windows + min(G, M) segments, each cut into
+  // at most 128 / TM chunks
+  const int64_t n_tiles = (N + bnr - 1) / bnr;
+  const int64_t chunks = (windows + (G < M ? G : M)) * nh;
+  const int64_t units = n_tiles * chunks;
+  const int grid = bsg_forced_grid(0, static_cast<int>(units < dev->sm_count ? units : dev->sm_count));
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (nh == 1)
+    bsg::fp8s::bsg_fp8_swap_kernel<<<grid, bsg::fp8s::THREADS, bsg::fp8s::smem_bytes<1>(), cs>>>(p);
+  else
+    bsg::fp8s::bsg_fp8_swap_n256_kernel<<<grid, bsg::fp8s::THREADS, bsg::fp8s::smem_bytes<2>(), cs>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the fp8 swapped kernel");
+  return BSG_OK;
+}
+
+// tactic 0: one SM per 128 x 256 tile; tactic 1: an SM pair per 256 x 256 tile (cta_group::2);
+// tactics 2, 3: fp8_swap_launch
 bsg_status fp8_launch(DeviceState* dev, const void* A, const void* B, const float* a_scale, const float* b_scale,
                       const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G,
                       bsg_stream_t stream, int tactic) {
+  if (tactic == 2 || tactic == 3)
+    return fp8_swap_launch(dev, A, B, a_scale, b_scale, m_indices, C, M, N, K, G, stream, tactic);
   bsg_status st;
   const int cg = tactic == 1 ? 2 : 1;
 

@@ -14,6 +14,12 @@
 //     num_waves  = ceil(units / (sm_count / cluster_size))
 //     throughput = the tile's sustained fraction of the FP8 / FP4 tensor peak measured on the
 //                  prefill workloads (the table below); the exhaustive sweep re-measures it
+// Operand-swapped FP8 tactics (swap = 1: B rows are the MMA's 128-row operand, a chunk of at most
+// tok tokens its N operand): the row tile is a token chunk,
+//     m_eff = M / (chunks * tok),  chunks = segments * ceil(M / segments / tok)
+// and tile_n is the unit's width in output columns.  The MMA is 16 * ceil(tokens / 16) wide, but a
+// unit's time was measured to depend on its K blocks, not on its token count (the per-K-block work
+// of the single issuing thread dominates when the MMAs are small), so m_eff charges the whole chunk.
 // The sweep over all tactics is what validates the ranking.
 #include <cmath>
 #include <cstdio>
@@ -29,21 +35,24 @@ namespace {
 
 struct Tactic {
   const char* name;
-  int tile_m;
+  int tile_m;      // rows per tile; for swap tactics the token chunk (tok)
   int tile_n;
   int cta_group;
   int cga_n;
   double throughput;
+  int swap;
 };
 
 // FP8 and NVFP4 tactic tables (kind 0 and 1).  Only tactics that exist as kernels are listed.
 const Tactic kFp8[] = {
-    {"fp8_1sm_m128_n256_s4", 128, 256, 1, 1, 0.47},
-    {"fp8_2sm_m256_n256_s6", 256, 256, 2, 1, 0.45},
+    {"fp8_1sm_m128_n256_s4", 128, 256, 1, 1, 0.47, 0},
+    {"fp8_2sm_m256_n256_s6", 256, 256, 2, 1, 0.45, 0},
+    {"fp8_swapab_1sm_n128_t128_s6", 128, 128, 1, 1, 0.24, 1},
+    {"fp8_swapab_1sm_n256_t64_s5", 64, 256, 1, 1, 0.23, 1},
 };
 const Tactic kNvfp4[] = {
-    {"nvfp4_1sm_m128_n256_s4", 128, 256, 1, 1, 0.52},
-    {"nvfp4_2sm_m256_n256_s5", 256, 256, 2, 1, 0.58},
+    {"nvfp4_1sm_m128_n256_s4", 128, 256, 1, 1, 0.52, 0},
+    {"nvfp4_2sm_m256_n256_s5", 256, 256, 2, 1, 0.58, 0},
 };
 
 const Tactic* table(int kind, int* n) {
@@ -132,9 +141,15 @@ double bsg_tactic_score(int kind, int tactic, int64_t M, int64_t N, int64_t K, i
   if (!tt || tactic < 0 || tactic >= n || M <= 0 || N <= 0 || G <= 0 || sm_count <= 0) return 0.0;
   const Tactic& t = tt[tactic];
   const BsgUnitEstimate est = bsg_estimate_units(M, G);
-  const double row_tiles = static_cast<double>(t.cta_group == 2 ? est.pairs : est.segments);
+  double row_tiles = static_cast<double>(t.cta_group == 2 ? est.pairs : est.segments);
   const double tiles_n = std::ceil(static_cast<double>(N) / t.tile_n);
-  const double m_eff = static_cast<double>(M) / (row_tiles * t.tile_m);
+  double m_eff = static_cast<double>(M) / (row_tiles * t.tile_m);
+  if (t.swap) {
+    const double seg = static_cast<double>(est.segments);
+    row_tiles = seg * std::ceil(std::ceil(static_cast<double>(M) / seg) / t.tile_m);
+    m_eff = static_cast<double>(M) / (row_tiles * t.tile_m);
+    if (m_eff > 1.0) m_eff = 1.0;
+  }
   const double n_eff = static_cast<double>(N) / (tiles_n * t.tile_n);
   const int cluster = t.cta_group * t.cga_n;
   const double units = row_tiles * tiles_n;

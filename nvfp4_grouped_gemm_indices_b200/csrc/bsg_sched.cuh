@@ -130,13 +130,15 @@ __device__ __forceinline__ int routed_expert(const int* __restrict__ m_indices, 
 // same expert are paired -- a run spanning several windows gives pairs of consecutive windows -- and
 // a segment without a partner is paired with an empty half (rows [0, 0): computed, never stored).
 // Cluster c of P/2 takes pair-units c, c + P/2, ...; CTA rank r of the pair receives half r.
+// TOK < 128 (PAIR = false only): a segment longer than TOK rows is cut into consecutive chunks of at
+// most TOK rows, each its own row tile (the operand-swapped kernel, whose token tile is TOK wide).
 constexpr int kScanBatch = 4;
 
 struct Seg {
   int row0, lo, hi, g;
 };
 
-template <int Q, int BN, bool PAIR>
+template <int Q, int BN, bool PAIR, int TOK = 128>
 __device__ void run_scheduler(UnitQueue<Q>& q, const int* __restrict__ m_indices, int M, int G, int n_tiles,
                               int n_group, const WaitCtx& wctx, int debug_mode) {
   if (debug_mode == kDebugWithholdSchedule) return;
@@ -212,7 +214,7 @@ __device__ void run_scheduler(UnitQueue<Q>& q, const int* __restrict__ m_indices
           emask[j] = __ballot_sync(FULL, is_end);
           nseg += __popc(smask[j]);
         }
-        if (!PAIR) {
+        if (!PAIR && TOK >= 128) {
           // every segment is a unit: skip the window in one step when this CTA owns none of it
           const long long units_here = static_cast<long long>(nseg) * tiles;
           if (next >= first + units_here) {
@@ -236,7 +238,16 @@ __device__ void run_scheduler(UnitQueue<Q>& q, const int* __restrict__ m_indices
           sg.hi = row0 + 32 * je + be + 1;
           sg.g = __shfl_sync(FULL, gsel, bs);
           if (!PAIR) {
-            if (!emit(sg, nullptr, t0, tiles)) alive = false;
+            if constexpr (TOK >= 128) {
+              if (!emit(sg, nullptr, t0, tiles)) alive = false;
+            } else {
+              for (int c = sg.lo; c < sg.hi && alive; c += TOK) {
+                Seg part = sg;
+                part.lo = c;
+                part.hi = min(sg.hi, c + TOK);
+                if (!emit(part, nullptr, t0, tiles)) alive = false;
+              }
+            }
           } else if (have_pending && pending.g == sg.g) {
             if (!emit(pending, &sg, t0, tiles)) alive = false;
             have_pending = false;

@@ -1,6 +1,7 @@
 """CPU-side checks of the C ABI: the library loads without a GPU, exports every function
 include/bsg.h declares, rejects bad arguments on the host (launching nothing), and its chooser
 ranks tactics by the page's score."""
+import math
 import os
 import re
 
@@ -144,10 +145,29 @@ def test_chooser_score_follows_the_page_formula(lib):
         s1 = bsg.bsg_tactic_score(0, 1, 8192, 4096, 7168, 8, 148)
         waves1 = -(-(pairs * 16) // 74)
         assert abs(s1 - (8192 / (pairs * 256)) * thr[t1] * 1.05 / (waves1 * 256)) < 1e-15
-        # a skewed, tiny-M routing over many experts leaves 2-SM tiles half empty: one SM wins
-        assert bsg.bsg_choose_tactic(0, 512, 4096, 7168, 64, 148) == 0
-        # with the measured tile throughputs the one-SM tile wins the prefill shape as well
+        # with the measured tile throughputs the one-SM tile wins the prefill shape
         assert bsg.bsg_choose_tactic(0, 8192, 4096, 7168, 8, 148) == 0
+    names = [bsg.bsg_tactic_name(0, t) for t in range(bsg.bsg_num_tactics(0))]
+    swaps = [t for t, nm in enumerate(names) if "swapab" in nm]
+    if swaps:
+        # operand-swapped tiles: the row tile is a chunk of at most `tok` tokens of one segment, charged
+        # in full.  M=512 over 64 experts: 4 windows + 63 = 67 segments of ~8 tokens -> 67 chunks
+        for t in swaps:
+            nm = names[t]
+            tile_n = int(nm.split("_n")[1].split("_")[0])
+            tok = int(nm.split("_t")[1].split("_")[0])
+            chunks = 67 * math.ceil(math.ceil(512 / 67) / tok)
+            m_eff = 512 / (chunks * tok)
+            waves = -(-(chunks * -(-4096 // tile_n)) // 148)
+            s_t = bsg.bsg_tactic_score(0, t, 512, 4096, 7168, 64, 148)
+            ratio = s_t / (m_eff / (waves * tile_n))   # = the tactic's throughput entry
+            assert 0.1 < ratio < 1.0, (nm, ratio)
+        # measured: the row tile streams the decode shape fastest, and the prefill shape too
+        assert bsg.bsg_choose_tactic(0, 512, 4096, 7168, 64, 148) == 0
+        assert bsg.bsg_choose_tactic(0, 8192, 4096, 7168, 8, 148) not in swaps
+        # the small 4-expert shape (runs of ~128 rows, 256 columns) fills two swapped units per segment
+        # where the row tile has one: the swapped 128-column tile ranks first (measured: a tie)
+        assert bsg.bsg_choose_tactic(0, 512, 256, 512, 4, 148) == swaps[0]
     assert bsg.bsg_tactic_score(0, 99, 1, 64, 128, 1, 148) == 0.0
 
 
