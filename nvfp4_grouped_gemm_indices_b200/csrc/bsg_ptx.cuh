@@ -1,5 +1,5 @@
 // bsg_ptx.cuh -- thin inline-PTX wrappers for the sm_100a features the kernels use:
-// mbarriers (with bounded waits), TMA tensor loads, tcgen05 (TMEM alloc, MMA, commit, copy, load)
+// mbarriers (with bounded waits), TMA tensor loads, tcgen05 (TMEM alloc, MMA, commit, load, store)
 // and the shared-memory matrix descriptors of the 5th-generation tensor cores.
 #pragma once
 
@@ -114,11 +114,6 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
-// Generic-proxy shared-memory writes -> visible to the async proxy (tcgen05.cp / TMA store).
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // ---------------------------------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_result, uint32_t ncols) {
@@ -174,11 +169,6 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
                : "memory");
 }
 
-// Shared memory (32 rows x 16 bytes) -> TMEM (lanes 0..31 of every lane quarter, 4 columns).
-__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t s_desc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
-}
-
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 16 consecutive 32-bit columns (lane i of the warp gets TMEM lane base+i).
@@ -232,16 +222,6 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
   return d;
 }
 
-// Descriptor of a dense, unswizzled [rows x 16 B] block (scale factors for tcgen05.cp).
-__device__ __forceinline__ uint64_t sdesc_sf(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-  d |= static_cast<uint64_t>(0) << 16;                    // leading byte offset: one core matrix in K
-  d |= static_cast<uint64_t>(128 >> 4) << 32;             // 8-row core matrices, 128 B apart
-  d |= static_cast<uint64_t>(1) << 46;
-  return d;                                               // layout 0: no swizzle
-}
-
 // Instruction descriptor, kind::f8f6f4: D fp32, A = B = E4M3, both K-major, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_f8f6f4_e4m3(int M, int N) {
   return (1u << 4)                       // D format fp32
@@ -255,16 +235,6 @@ __host__ __device__ constexpr uint32_t idesc_mxf4nvf4(int M, int N) {
          | (static_cast<uint32_t>(N >> 3) << 17)
          | (0u << 23)                       // scale format UE4M3
          | (static_cast<uint32_t>(M >> 4) << 24);
-}
-
-// Per-warpgroup register reallocation (all 4 warps of the warpgroup execute it).
-template <int N>
-__device__ __forceinline__ void setmaxnreg_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void setmaxnreg_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ---------------------------------------------------------------------------------- CTA pairs
@@ -362,26 +332,6 @@ __device__ __forceinline__ void tc_commit_pair_multicast(uint64_t* bar, uint16_t
           smem_u32(bar)),
       "h"(cta_mask)
       : "memory");
-}
-
-// Hardware named barrier over `nthreads` threads (a multiple of 32) of the CTA; id 1..15.
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// Named barrier that also ORs a predicate over the participating threads: every thread gets the same
-// answer, so a group can leave a loop together (no thread is left waiting on the barrier).
-__device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.or.pred p, %2, %3, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(r)
-      : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
 }
 
 // ------------------------------------------------------------------------------------------ misc
