@@ -15,7 +15,8 @@ Formats (bit layouts are those of the OCP 8-bit / 4-bit floating-point formats):
 Quantisation recipes (the five workloads of the benchmark):
 
 * FP8: per 1x128 K block of A and per 128x128 block of B[g]: ``scale = amax / 448`` (fp32),
-  ``code = e4m3_rne_satfinite(x / scale)``; an all-zero block gets scale 0 and zero codes.
+  ``code = e4m3_rne_satfinite(x / scale)`` with the quotient one correctly rounded fp32 division;
+  an all-zero block gets scale 0 and zero codes.
 * NVFP4: ``gs = amax(tensor) / (448 * 6)``; per 16 K elements ``s = ue4m3_rne((amax16 / 6) / gs)``;
   ``code = e2m1_rne_satfinite(x / (s * gs))``; ``alpha[g] = gs_A * gs_B[g]`` (B's global scale is
   taken per expert, each B[g] being its own weight tensor).
@@ -100,10 +101,10 @@ def quant_fp8_rows(x: np.ndarray):
     xb = x.reshape(R, K // 128, 128)
     amax = np.abs(xb).max(axis=-1).astype(np.float32)
     scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
-    inv = np.where(scale > 0, np.float32(1.0) / np.where(scale > 0, scale, np.float32(1.0)),
-                   np.float32(0.0)).astype(np.float32)
-    q = (xb * inv[..., None]).astype(np.float32)
-    return e4m3_encode(q).reshape(R, K), scale
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    q = (xb / safe[..., None]).astype(np.float32)          # one correctly rounded fp32 division
+    codes = np.where((scale > 0)[..., None], e4m3_encode(q), np.uint8(0))
+    return codes.astype(np.uint8).reshape(R, K), scale
 
 
 def quant_fp8_blocks(w: np.ndarray):
@@ -117,9 +118,10 @@ def quant_fp8_blocks(w: np.ndarray):
         blk = w[nb * 128:(nb + 1) * 128].reshape(-1, K // 128, 128)
         amax = np.abs(blk).max(axis=(0, 2)).astype(np.float32)
         s = (amax / np.float32(E4M3_MAX)).astype(np.float32)
-        inv = np.where(s > 0, np.float32(1.0) / np.where(s > 0, s, np.float32(1.0)), np.float32(0.0))
-        q = (blk * inv.astype(np.float32)[None, :, None]).astype(np.float32)
-        codes[nb * 128:(nb + 1) * 128] = e4m3_encode(q).reshape(-1, K)
+        safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+        q = (blk / safe[None, :, None]).astype(np.float32)
+        c = np.where((s > 0)[None, :, None], e4m3_encode(q), np.uint8(0)).astype(np.uint8)
+        codes[nb * 128:(nb + 1) * 128] = c.reshape(-1, K)
         scale[nb] = s
     return codes, scale
 
@@ -145,10 +147,9 @@ def quant_nvfp4(x: np.ndarray, gs: np.float32, chunk_rows: int = 4096):
             s_code = np.zeros(amax16.shape, dtype=np.uint8)
         s_val = e4m3_decode(s_code).astype(np.float32)
         denom = (s_val * gs).astype(np.float32)
-        inv = np.where(denom > 0, np.float32(1.0) / np.where(denom > 0, denom, np.float32(1.0)),
-                       np.float32(0.0)).astype(np.float32)
-        q = (xb * inv[..., None]).astype(np.float32)
-        codes = e2m1_encode(q).reshape(-1, K)
+        safe = np.where(denom > 0, denom, np.float32(1.0)).astype(np.float32)
+        q = (xb / safe[..., None]).astype(np.float32)       # one correctly rounded fp32 division
+        codes = np.where((denom > 0)[..., None], e2m1_encode(q), np.uint8(0)).astype(np.uint8).reshape(-1, K)
         packed[r0:r0 + chunk_rows] = pack_e2m1(codes)
         sf[r0:r0 + chunk_rows] = s_code
     return packed, sf

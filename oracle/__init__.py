@@ -18,6 +18,9 @@ Functions (all numpy in, numpy out):
 * ``enc_e4m3``, ``enc_e2m1``, ``quant_fp8_rows``, ``quant_nvfp4_rows`` -- the step before the GEMM:
   BF16 activations (optionally gathered by a row map, the MoE expand) quantised into the GEMM's
   input formats, from the format definitions (RNE, saturating) with every step in IEEE fp32.
+* ``moe_permute(expert_ids, G)`` -- the MoE expand permutation that makes each expert's rows one
+  contiguous run (the expanded input rows of the ONNX Runtime page, section 1): a plain stable
+  counting sort of the (token, choice) entries by expert, with the inverse map.
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py`` (decode tables, exact
 integer grids, grouped == dense, exact rational brute force, fp64 library matmul, the printed CTA
@@ -58,6 +61,8 @@ def lib():
         L.bsg_oracle_quant_fp8_rows.argtypes = [p, p, i64, i64, i64, p, p]
         L.bsg_oracle_quant_nvfp4_rows.restype = ctypes.c_int
         L.bsg_oracle_quant_nvfp4_rows.argtypes = [p, p, ctypes.c_float, i64, i64, i64, p, p]
+        L.bsg_oracle_moe_permute.restype = ctypes.c_int
+        L.bsg_oracle_moe_permute.argtypes = [p, i64, i64, i64, p, p, p, p]
         L.bsg_oracle_max_threads.restype = ctypes.c_int
         L.bsg_oracle_set_threads.argtypes = [ctypes.c_int]
         _lib = L
@@ -156,7 +161,8 @@ def enc_e2m1(x):
 
 def quant_fp8_rows(X_bf16_bits, M=None, src_rows=None, A=None, scale=None):
     """Activation quantisation to the FP8 GEMM's A operand: per 1 x 128 block, scale = amax/448,
-    code = e4m3_rne_satfinite(x * (1 / scale)) in fp32 (one reciprocal per block).  X: uint16 bf16 bits [M_in, K]; output row m is
+    code = e4m3_rne_satfinite(x / scale), the quotient one correctly rounded fp32 division per
+    element; a zero block gets zero codes.  X: uint16 bf16 bits [M_in, K]; output row m is
     input row src_rows[m] (or m).  Returns (A uint8 [M, K], scale f32 [M, K/128]); rows whose
     source is out of range keep the initial contents of A / scale (default 0xFF / NaN)."""
     L = lib()
@@ -176,8 +182,8 @@ def quant_fp8_rows(X_bf16_bits, M=None, src_rows=None, A=None, scale=None):
 
 def quant_nvfp4_rows(X_bf16_bits, gs, M=None, src_rows=None, A=None, sf=None):
     """Activation quantisation to the NVFP4 GEMM's A operand with global scale gs: per 1 x 16
-    block, s = ue4m3_rne_satfinite((amax/6)/gs), code = e2m1_rne_satfinite(x * (1 / (dec(s) * gs))),
-    all in fp32.  Returns (A uint8 [M, K/2] packed, low nibble = lower K; sf uint8 [M, K/16])."""
+    block, s = ue4m3_rne_satfinite((amax/6)/gs), code = e2m1_rne_satfinite(x / (dec(s) * gs)),
+    every step one correctly rounded fp32 operation (one division per element).  Returns (A uint8 [M, K/2] packed, low nibble = lower K; sf uint8 [M, K/16])."""
     L = lib()
     X = np.ascontiguousarray(X_bf16_bits, dtype=np.uint16)
     M_in, K = X.shape
@@ -191,6 +197,27 @@ def quant_nvfp4_rows(X_bf16_bits, gs, M=None, src_rows=None, A=None, sf=None):
     if rc != 0:
         raise ValueError("oracle quant_nvfp4_rows: invalid sizes")
     return A, sf
+
+
+def moe_permute(expert_ids, G):
+    """The MoE expand permutation: a stable counting sort of the (token, choice) entries of
+    expert_ids [T, top_k] (token-major) by expert.  Returns (src_rows int32 [T*top_k], m_indices
+    int32 [T*top_k], dst_rows int32 [T, top_k], expert_offsets int32 [G+1]); entries whose expert
+    is outside [0, G) are dropped (dst_rows -1) and the unused tail positions hold -1."""
+    L = lib()
+    e = np.ascontiguousarray(expert_ids, dtype=np.int32)
+    if e.ndim != 2:
+        raise ValueError("expert_ids must be [T, top_k]")
+    T, top_k = e.shape
+    n = T * top_k
+    src = np.empty(n, np.int32)
+    mi = np.empty(n, np.int32)
+    dst = np.empty((T, top_k), np.int32)
+    off = np.empty(G + 1, np.int32)
+    rc = L.bsg_oracle_moe_permute(_ptr(e), T, top_k, int(G), _ptr(src), _ptr(mi), _ptr(dst), _ptr(off))
+    if rc != 0:
+        raise ValueError("oracle moe_permute: invalid sizes")
+    return src, mi, dst, off
 
 
 def set_threads(n):

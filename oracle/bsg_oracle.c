@@ -33,6 +33,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 #ifdef _OPENMP
 #include <omp.h>
@@ -205,17 +206,16 @@ int bsg_oracle_nvfp4(const uint8_t* A, const uint8_t* B, const uint8_t* sfa, con
  * contiguous runs; row m of the output is row src_rows[m] of the input).  Written from the format
  * definitions and the quantisation recipe of the two GEMMs' inputs:
  *
- *   FP8, per 1 x 128 block:  scale = amax / 448;  code = e4m3_rne_satfinite(x * (1 / scale))
+ *   FP8, per 1 x 128 block:  scale = amax / 448;  code = e4m3_rne_satfinite(x / scale)
  *   NVFP4, per 1 x 16 block, global scale gs:
- *       s = ue4m3_rne_satfinite((amax16 / 6) / gs);  code = e2m1_rne_satfinite(x * (1 / (dec(s) * gs)))
+ *       s = ue4m3_rne_satfinite((amax16 / 6) / gs);  code = e2m1_rne_satfinite(x / (dec(s) * gs))
  *
- * Each element is multiplied by the reciprocal of its block's scale, computed once per block (the
- * pages fix the scale, not how the division by it is carried out; one reciprocal per block and a
- * product per element is how block quantisers are written).  Every operation is the IEEE fp32 one
- * (division, reciprocal and product correctly rounded, no fused multiply-add), because the quantised
- * code is an integer decided in fp32 on the GPU as well.  A block whose scale is zero gets all-zero
- * codes.  The encoders round to the nearest representable value, ties to the even code, and
- * saturate at the largest finite magnitude (448, 6).
+ * Every operation is the IEEE fp32 one (each division and product correctly rounded, no fused
+ * multiply-add): the quotient x / scale is formed once per element as a single correctly rounded fp32
+ * division, and the encoder then rounds that fp32 value to the code.  The code is an integer decided
+ * in fp32, so a GPU that reaches the same fp32 quotient reaches the same code.  A block whose scale is
+ * zero (every element zero) gets all-zero codes.  The encoders round to the nearest representable
+ * value, ties to the even code, and saturate at the largest finite magnitude (448, 6).
  */
 
 /* fp32 -> E4M3 (FN) code: RNE, saturating at +-448; NaN -> 0x7F with the sign. */
@@ -282,10 +282,13 @@ int bsg_oracle_quant_fp8_rows(const uint16_t* X, const int32_t* src_rows, int64_
       }
       volatile float s = amax / 448.0f;
       scale[m * KB + kb] = s;
-      volatile float inv = (s > 0.0f) ? 1.0f / s : 0.0f;
       for (int64_t k = 0; k < 128; ++k) {
+        if (!(s > 0.0f)) {               /* zero block: zero codes */
+          A[m * K + kb * 128 + k] = 0;
+          continue;
+        }
         float v = bf16_bits_to_f32(x[kb * 128 + k]);
-        volatile float q = v * inv;
+        volatile float q = v / s;
         A[m * K + kb * 128 + k] = bsg_oracle_enc_e4m3(q);
       }
     }
@@ -315,17 +318,78 @@ int bsg_oracle_quant_nvfp4_rows(const uint16_t* X, const int32_t* src_rows, floa
       uint8_t sc = bsg_oracle_enc_e4m3(t2);
       sf[m * KS + j] = sc;
       volatile float denom = (float)bsg_oracle_dec_e4m3(sc) * gs;
-      volatile float inv = (denom > 0.0f) ? 1.0f / denom : 0.0f;
       uint8_t codes[16];
       for (int64_t k = 0; k < 16; ++k) {
+        if (!(denom > 0.0f)) {           /* zero scale: zero codes */
+          codes[k] = 0;
+          continue;
+        }
         float v = bf16_bits_to_f32(x[j * 16 + k]);
-        volatile float q = v * inv;
+        volatile float q = v / denom;
         codes[k] = bsg_oracle_enc_e2m1(q);
       }
       for (int64_t k = 0; k < 16; k += 2)
         A[m * (K / 2) + (j * 16 + k) / 2] = (uint8_t)(codes[k] | (codes[k + 1] << 4));
     }
   }
+  return 0;
+}
+
+/* ---------------------------------------------------------------- MoE expand permutation ---- */
+
+/*
+ * The MoE "expand" that precedes the activation quantiser and the grouped GEMM (the expanded input
+ * rows of the ONNX Runtime page, "[onnxruntime] ONNX Runtime: Blackwell (SM120+)에서 NVFP4 QMoE를 위한
+ * 네이티브 FP4xFP4 Prefill 최적화", section 1): every token t has top_k expert choices
+ * expert_ids[t, k]; the T * top_k (token, choice) entries are laid out expert by expert so that each
+ * expert's rows form one contiguous run of the GEMM's A.  Written as a plain stable counting sort of
+ * the entries, taken in token-major order i = t * top_k + k, by their expert:
+ *
+ *   count[g]          = number of entries with expert g                 (g in [0, G))
+ *   expert_offsets[g] = count[0] + ... + count[g - 1];  expert_offsets[G] = entries placed
+ *   entry i with expert g in [0, G) goes to the next free position p of g's run, in increasing i:
+ *       src_rows[p] = t,  m_indices[p] = g,  dst_rows[i] = p
+ *   an entry whose expert is outside [0, G) is dropped: dst_rows[i] = -1
+ *   positions p in [expert_offsets[G], T * top_k) hold src_rows[p] = m_indices[p] = -1
+ *
+ * so the GEMM skips those rows and the quantiser leaves them untouched.  dst_rows is the inverse
+ * map a later combine needs (row dst_rows[t, k] of the GEMM's output belongs to token t, choice k).
+ * Returns 0, or -1 for an invalid size.
+ */
+int bsg_oracle_moe_permute(const int32_t* expert_ids, int64_t T, int64_t top_k, int64_t G, int32_t* src_rows,
+                           int32_t* m_indices, int32_t* dst_rows, int32_t* expert_offsets) {
+  if (T < 0 || top_k < 1 || G < 1) return -1;
+  const int64_t n = T * top_k;
+  int64_t* next = (int64_t*)calloc((size_t)G, sizeof(int64_t));
+  if (!next) return -1;
+  for (int64_t i = 0; i < n; ++i) {
+    const int32_t g = expert_ids[i];
+    if (g >= 0 && g < G) next[g] += 1;
+  }
+  int64_t run = 0;
+  for (int64_t g = 0; g < G; ++g) {
+    const int64_t c = next[g];
+    expert_offsets[g] = (int32_t)run;
+    next[g] = run;
+    run += c;
+  }
+  expert_offsets[G] = (int32_t)run;
+  for (int64_t i = 0; i < n; ++i) {
+    const int32_t g = expert_ids[i];
+    if (g >= 0 && g < G) {
+      const int64_t p = next[g]++;
+      src_rows[p] = (int32_t)(i / top_k);
+      m_indices[p] = g;
+      dst_rows[i] = (int32_t)p;
+    } else {
+      dst_rows[i] = -1;
+    }
+  }
+  for (int64_t p = run; p < n; ++p) {
+    src_rows[p] = -1;
+    m_indices[p] = -1;
+  }
+  free(next);
   return 0;
 }
 

@@ -6,6 +6,9 @@ the arithmetic fix, independently of the oracle's own code:
   the nearer one; magnitudes past the largest finite value saturate;
 * the quantisers agree bit for bit with the input generators' vectorised implementation (numpy
   and the library's float8 type), which shares nothing with the oracle;
+* on inputs built so that the correctly rounded quotient x / scale and the product x * (1 / scale)
+  round to different codes, the codes are those of the quotient (one IEEE fp32 division per
+  element, the quantiser as the format recipe writes it);
 * each block's largest element lands on +-448 (FP8) and dequantised values sit within half a step
   of the input; a zero block gives zero scale and zero codes;
 * gathering rows first equals quantising the gathered matrix (the MoE expand).
@@ -90,7 +93,8 @@ def test_fp8_rows_match_generator_and_pin_the_block_maximum():
     dq = oracle.dec_e4m3(A).reshape(M, K // 128, 128) * s[..., None]
     q = blocks / s[..., None]
     step = np.where(np.abs(q) < 2.0 ** -6, 2.0 ** -9, 2.0 ** (np.floor(np.log2(np.maximum(np.abs(q), 1e-30))) - 3))
-    assert np.all(np.abs(dq - blocks) <= 0.5 * step * s[..., None] * (1 + 1e-5))
+    # |dec(code) - x/s| <= half a step + the quotient's own rounding (2^-24 |q|, |q| < 16 steps)
+    assert np.all(np.abs(dq - blocks) <= 0.5 * step * s[..., None] * (1 + 2.0 ** -19))
 
 
 def test_nvfp4_rows_match_generator():
@@ -133,3 +137,31 @@ def test_gather_equals_quantising_the_gathered_rows():
     A4_ref, sf_ref = oracle.quant_nvfp4_rows(xb[src[ok]], np.float32(0.01))
     assert np.array_equal(A4[ok], A4_ref) and np.array_equal(sf[ok], sf_ref)
     assert np.all(A4[~ok] == 0xFF) and np.all(sf[~ok] == 0xFF)
+
+
+def test_fp8_quotient_not_reciprocal_on_adversarial_inputs():
+    from adversarial import fp8_rows
+    xb, adv = fp8_rows(n_blocks=48, seed=8)
+    assert adv.sum() >= 200
+    x = bf16_bits_to_f32(xb)
+    A, s = oracle.quant_fp8_rows(xb)
+    blocks = x.reshape(1, -1, 128)
+    sb = s[..., None]
+    div = W.e4m3_encode((blocks / sb).astype(np.float32)).reshape(A.shape)        # IEEE fp32 division
+    rcp = W.e4m3_encode((blocks * (np.float32(1) / sb)).astype(np.float32)).reshape(A.shape)
+    assert np.array_equal(A, div)
+    assert np.all(A[adv] != rcp[adv])
+
+
+def test_nvfp4_quotient_not_reciprocal_on_adversarial_inputs():
+    from adversarial import nvfp4_cases
+    cases = nvfp4_cases(n=10, seed=9)
+    assert len(cases) == 10
+    for gs, xb, adv in cases:
+        x = bf16_bits_to_f32(xb).reshape(-1, 16)
+        A, sf = oracle.quant_nvfp4_rows(xb, gs)
+        d = (oracle.dec_e4m3(sf.reshape(-1)).astype(np.float32) * np.float32(gs)).astype(np.float32)[:, None]
+        div = W.pack_e2m1(W.e2m1_encode((x / d).astype(np.float32)).reshape(1, -1))
+        rcp_codes = W.e2m1_encode((x * (np.float32(1) / d)).astype(np.float32)).reshape(1, -1)
+        assert np.array_equal(A, div)
+        assert np.all(W.unpack_e2m1(A)[adv] != rcp_codes[adv])
