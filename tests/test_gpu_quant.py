@@ -111,3 +111,64 @@ def test_quantise_then_gemm_matches_the_oracle_chain():
     assert np.array_equal(A.cpu().numpy(), A_ref)
     ref, _ = oracle.fp8_grouped(A_ref, w.B, s_ref, w.b_scale, m_indices, T, N, K, G)
     compare(C.view(torch.int16).cpu().numpy().view(np.uint16), ref, routed_mask(w))
+
+
+def test_fp8_adversarial_quotients_bit_exact():
+    """Elements whose correctly rounded quotient x / scale and product x * (1 / scale) round to
+    different E4M3 codes (built in numpy by tests/adversarial.py): the kernel must give the
+    quotient's code, as the oracle does."""
+    from adversarial import fp8_rows
+    xb, adv = fp8_rows(n_blocks=64, seed=31)
+    rows = np.repeat(xb, 3, axis=0)                      # three rows: every lane position is exercised
+    rows[1] = np.roll(xb[0], 128)
+    rows[2] = np.roll(xb[0], 1024)
+    M, K = rows.shape
+    xt = torch.from_numpy(rows.view(np.int16).copy()).view(torch.bfloat16)
+    A, s = bsg.quantize_fp8_rows(xt.cuda())
+    torch.cuda.synchronize()
+    A_ref, s_ref = oracle.quant_fp8_rows(rows)
+    assert adv.sum() >= 150
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(A.cpu().numpy(), A_ref)
+
+
+def test_nvfp4_adversarial_quotients_bit_exact():
+    from adversarial import nvfp4_cases
+    cases = nvfp4_cases(n=16, seed=32)
+    assert len(cases) == 16
+    for gs, xb, adv in cases:
+        M, K = xb.shape
+        xt = torch.from_numpy(xb.view(np.int16).copy()).view(torch.bfloat16)
+        A, sf = bsg.quantize_nvfp4_rows(xt.cuda(), torch.tensor([gs], dtype=torch.float32, device="cuda"))
+        torch.cuda.synchronize()
+        A_ref, sf_ref = oracle.quant_nvfp4_rows(xb, gs)
+        assert np.array_equal(sf.cpu().numpy(), sf_ref)
+        assert np.array_equal(A.cpu().numpy(), A_ref), f"gs {gs!r}"
+
+
+def test_tiny_scales_and_signed_zeros():
+    """Blocks so small that the fp32 reciprocal of their scale overflows, and blocks of signed zeros
+    (scale 0: every code is 0, the sign of a zero input included)."""
+    K = 512
+    rows = np.zeros((4, K), np.uint16)
+    rng = np.random.default_rng(40)
+    tiny = rng.integers(0x0001, 0x0080, K).astype(np.uint16) | (rng.integers(0, 2, K).astype(np.uint16) << 15)
+    rows[0] = tiny                                        # bf16 subnormals: amax / 448 is an fp32 subnormal
+    rows[1, :128] = 0x8000                                # -0 everywhere in block 0
+    rows[1, 128:] = (rng.standard_normal(K - 128).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    rows[2, ::2] = 0x8000                                 # -0 between normal values
+    rows[2, 1::2] = 0x3F80
+    rows[3] = (rng.standard_normal(K).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    xt = torch.from_numpy(rows.view(np.int16).copy()).view(torch.bfloat16)
+    A, s = bsg.quantize_fp8_rows(xt.cuda())
+    torch.cuda.synchronize()
+    A_ref, s_ref = oracle.quant_fp8_rows(rows)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(A.cpu().numpy(), A_ref)
+    assert np.all(A_ref[1, :128] == 0)
+    for gs in (np.float32(1e-30), np.float32(1e-3), np.float32(7.5e-41)):
+        A4, sf = bsg.quantize_nvfp4_rows(xt.cuda(), torch.tensor([gs], dtype=torch.float32, device="cuda"))
+        torch.cuda.synchronize()
+        A4_ref, sf_ref = oracle.quant_nvfp4_rows(rows, gs)
+        assert np.array_equal(sf.cpu().numpy(), sf_ref), f"gs {gs!r}"
+        assert np.array_equal(A4.cpu().numpy(), A4_ref), f"gs {gs!r}"
