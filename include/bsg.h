@@ -15,6 +15,7 @@
 #ifndef BSG_H_
 #define BSG_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -91,13 +92,15 @@ bsg_status bsg_nvfp4_gemm(const void* A, const void* B, const void* sfa, const v
  *
  *   for every output row m with r = (src_rows ? src_rows[m] : m) in [0, M_in):
  *     FP8,   per 128-element block b:  a_scale[m,b] = amax / 448
- *                                      A[m,k] = e4m3(X[r,k] * (1 / a_scale[m,b]))
+ *                                      A[m,k] = e4m3(X[r,k] / a_scale[m,b])
  *     NVFP4, per 16-element block j:   sfa[m,j]   = ue4m3((amax / 6) / gs)
- *                                      A[m,k]     = e2m1(X[r,k] * (1 / (sfa[m,j] * gs)))
- *   amax is the largest |X[r,k]| of the block; every step is an IEEE fp32 operation (the reciprocal
- *   is taken once per block); e4m3 / e2m1 /
- *   ue4m3 round to the nearest value, ties to the even code, and saturate at 448 / 6 / 448; a zero
- *   block gets scale 0 and zero codes.  Output rows whose source is outside [0, M_in) are not written.
+ *                                      A[m,k]     = e2m1(X[r,k] / (sfa[m,j] * gs))
+ *   amax is the largest |X[r,k]| of the block; every step is an IEEE fp32 operation and each
+ *   quotient the correctly rounded fp32 division (the codes are those of one division per element);
+ *   e4m3 / e2m1 / ue4m3 round to the nearest value, ties to the even code, and saturate at 448 / 6 /
+ *   448 (the saturating conversion of the page "[sglang] ROCm 아키텍처별 최적화: 런타임 디스패치로 성능
+ *   극대화", section 1); a zero block gets scale 0 and zero codes.  Output rows whose source is
+ *   outside [0, M_in) are not written.
  *
  * X         bf16  [M_in, K]  activations (finite values), row-major, 16-byte aligned.
  * src_rows  int32 [M]        source row of each output row, or NULL (then M <= M_in, row m <- row m).
@@ -112,6 +115,40 @@ bsg_status bsg_quantize_fp8_rows(const void* X, const int32_t* src_rows, void* A
                                  int64_t M, int64_t K, bsg_stream_t stream);
 bsg_status bsg_quantize_nvfp4_rows(const void* X, const int32_t* src_rows, const float* global_scale, void* A,
                                    void* sfa, int64_t M_in, int64_t M, int64_t K, bsg_stream_t stream);
+
+/*
+ * MoE expand permutation -- the step before the quantiser: lay the routing entries out expert by
+ * expert so that each expert's rows form one contiguous run of the grouped GEMM's A (the expanded
+ * input rows of the ONNX Runtime page cited above, section 1).  A stable counting sort of the
+ * n = T * top_k entries i = t * top_k + k (token-major) by their expert g = expert_ids[i]:
+ *
+ *   expert_offsets[g] = number of entries with an expert below g;  expert_offsets[G] = entries placed
+ *   entry i with g in [0, G) takes the next position p of g's run, in increasing i:
+ *       src_rows[p] = t,  m_indices[p] = g,  dst_rows[i] = p
+ *   entry i with g outside [0, G) is dropped: dst_rows[i] = -1
+ *   positions p in [expert_offsets[G], n): src_rows[p] = m_indices[p] = -1
+ *
+ * so bsg_quantize_*_rows(X, src_rows, ..., M_in = T, M = n) gathers the expanded activations (it
+ * leaves the -1 rows untouched), the grouped GEMM takes m_indices as is (it skips the -1 rows), and
+ * a later combine finds the output row of token t's choice k at dst_rows[t, k].
+ *
+ * expert_ids      int32 [T, top_k]  routing choices (any value; those outside [0, G) are dropped).
+ * src_rows        int32 [n]         output: source token of each expanded row.
+ * m_indices       int32 [n]         output: expert of each expanded row, non-decreasing, then -1.
+ * dst_rows        int32 [T, top_k]  output: expanded row of each entry, or -1.
+ * expert_offsets  int32 [G + 1]     output: start of each expert's run; [G] = rows placed.
+ * workspace       device scratch of at least bsg_moe_permute_workspace_size() bytes, 16-byte
+ *                 aligned, owned by the caller; its contents need not be initialised and are
+ *                 overwritten.  Calls that share a workspace must not overlap on the GPU.
+ * Contract: T >= 1, 1 <= top_k <= 256, T * top_k <= 2^24, 1 <= G <= 4096; the int32 arrays 4-byte
+ *           aligned.  Asynchronous on `stream`; nothing is allocated.  Three kernel launches.
+ * bsg_moe_permute_workspace_size() writes the scratch size for (T, top_k, G) to *bytes (at most
+ * 16 MiB) or returns an error for sizes outside the contract; it touches no GPU.
+ */
+bsg_status bsg_moe_permute_workspace_size(int64_t T, int64_t top_k, int64_t G, size_t* bytes);
+bsg_status bsg_moe_permute(const int32_t* expert_ids, int64_t T, int64_t top_k, int64_t G, int32_t* src_rows,
+                           int32_t* m_indices, int32_t* dst_rows, int32_t* expert_offsets, void* workspace,
+                           size_t workspace_bytes, bsg_stream_t stream);
 
 /* Description of the last failure on the calling thread ("" if none).  The string stays valid until
  * the next bsg_* call on the same thread. */

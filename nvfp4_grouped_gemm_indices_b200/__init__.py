@@ -15,8 +15,10 @@ Convenience wrappers infer the sizes from torch tensors and allocate C when not 
     fp8_grouped_gemm(A, B, a_scale, b_scale, m_indices, out=None)
     nvfp4_gemm(A, B, sfa, sfb, alpha, m_indices, out=None)
 
-and the step before the GEMM (activation quantisation with an optional row gather)::
+and the steps before the GEMM (the MoE expand permutation, then activation quantisation with a row
+gather)::
 
+    moe_permute(expert_ids, G) -> (src_rows, m_indices, dst_rows, expert_offsets)
     quantize_fp8_rows(X, src_rows=None) -> (A, a_scale)
     quantize_nvfp4_rows(X, global_scale, src_rows=None) -> (A, sfa)
 """
@@ -47,7 +49,7 @@ EXPORTED = [
     "bsg_set_wait_timeout_ns", "bsg_num_tactics", "bsg_tactic_name", "bsg_choose_tactic",
     "bsg_tactic_score", "bsg_set_tactic", "bsg_set_max_ctas", "bsg_debug_set_fault", "bsg_version",
     "bsg_quantize_fp8_rows", "bsg_quantize_nvfp4_rows", "bsg_autotune_fp8", "bsg_autotune_nvfp4",
-    "bsg_autotune_clear",
+    "bsg_autotune_clear", "bsg_moe_permute_workspace_size", "bsg_moe_permute",
 ]
 
 
@@ -106,6 +108,10 @@ def load(path: Optional[str] = None):
     L.bsg_autotune_clear.argtypes = []
     L.bsg_quantize_nvfp4_rows.restype = i32
     L.bsg_quantize_nvfp4_rows.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    L.bsg_moe_permute_workspace_size.restype = i32
+    L.bsg_moe_permute_workspace_size.argtypes = [i64, i64, i64, ctypes.POINTER(ctypes.c_size_t)]
+    L.bsg_moe_permute.restype = i32
+    L.bsg_moe_permute.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     if path is None:
         _lib = L
     return L
@@ -159,6 +165,19 @@ def bsg_quantize_fp8_rows(X, src_rows, A, a_scale, M_in, M, K, stream=None):
 def bsg_quantize_nvfp4_rows(X, src_rows, global_scale, A, sfa, M_in, M, K, stream=None):
     _check(load().bsg_quantize_nvfp4_rows(_ptr(X), _ptr(src_rows), _ptr(global_scale), _ptr(A), _ptr(sfa),
                                           int(M_in), int(M), int(K), _stream(stream)))
+
+
+def bsg_moe_permute_workspace_size(T, top_k, G) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().bsg_moe_permute_workspace_size(int(T), int(top_k), int(G), ctypes.byref(n)))
+    return int(n.value)
+
+
+def bsg_moe_permute(expert_ids, T, top_k, G, src_rows, m_indices, dst_rows, expert_offsets, workspace,
+                    workspace_bytes, stream=None):
+    _check(load().bsg_moe_permute(_ptr(expert_ids), int(T), int(top_k), int(G), _ptr(src_rows), _ptr(m_indices),
+                                  _ptr(dst_rows), _ptr(expert_offsets), _ptr(workspace), int(workspace_bytes),
+                                  _stream(stream)))
 
 
 def bsg_autotune_fp8(A, B, a_scale, b_scale, m_indices, C, M, N, K, G, reps=20, stream=None) -> int:
@@ -242,6 +261,23 @@ def _need(t, dtype, name, dims=None):
         raise ValueError(f"{name} must have {dims} dimensions, got {t.dim()}")
 
 
+def _same_device(named, stream=None):
+    """Every tensor (and the stream, if given) must be on one CUDA device; returns that device.  The
+    library launches on the current device, so the wrappers make it current for the call."""
+    dev = None
+    for name, t in named:
+        if t is None:
+            continue
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device} but the other operands are on {dev}")
+    if stream is not None and not isinstance(stream, int) and hasattr(stream, "device"):
+        if stream.device != dev:
+            raise ValueError(f"stream is on {stream.device} but the operands are on {dev}")
+    return dev
+
+
 def fp8_grouped_gemm(A, B, a_scale, b_scale, m_indices, out=None, stream=None):
     """A uint8/float8 [M,K], B [G,N,K], a_scale f32 [M,K/128], b_scale f32 [G,ceil(N/128),K/128],
     m_indices int32 [M] (or None when G == 1).  Returns C bf16 [M,N] (unrouted rows of a fresh C
@@ -265,13 +301,16 @@ def fp8_grouped_gemm(A, B, a_scale, b_scale, m_indices, out=None, stream=None):
         _need(m_indices, torch.int32, "m_indices", 1)
         if m_indices.numel() != M:
             raise ValueError("m_indices must have M entries")
-    if out is None:
-        out = torch.zeros((M, N), dtype=torch.bfloat16, device=A8.device)
-    else:
+    if out is not None:
         _need(out, torch.bfloat16, "out", 2)
         if tuple(out.shape) != (M, N):
             raise ValueError(f"out must be [{M}, {N}]")
-    bsg_fp8_grouped_gemm(A8, B8, a_scale, b_scale, m_indices, out, M, N, K, G, stream)
+    dev = _same_device((("A", A8), ("B", B8), ("a_scale", a_scale), ("b_scale", b_scale),
+                        ("m_indices", m_indices), ("out", out)), stream)
+    with torch.cuda.device(dev):
+        if out is None:
+            out = torch.zeros((M, N), dtype=torch.bfloat16, device=dev)
+        bsg_fp8_grouped_gemm(A8, B8, a_scale, b_scale, m_indices, out, M, N, K, G, stream)
     return out
 
 
@@ -298,12 +337,37 @@ def nvfp4_gemm(A, B, sfa, sfb, alpha, m_indices, out=None, stream=None):
         _need(m_indices, torch.int32, "m_indices", 1)
         if m_indices.numel() != M:
             raise ValueError("m_indices must have M entries")
-    if out is None:
-        out = torch.zeros((M, N), dtype=torch.bfloat16, device=A.device)
-    else:
+    if out is not None:
         _need(out, torch.bfloat16, "out", 2)
-    bsg_nvfp4_gemm(A, B, sfa, sfb, alpha, m_indices, out, M, N, K, G, stream)
+        if tuple(out.shape) != (M, N):
+            raise ValueError(f"out must be [{M}, {N}]")
+    dev = _same_device((("A", A), ("B", B), ("sfa", sfa), ("sfb", sfb), ("alpha", alpha),
+                        ("m_indices", m_indices), ("out", out)), stream)
+    with torch.cuda.device(dev):
+        if out is None:
+            out = torch.zeros((M, N), dtype=torch.bfloat16, device=dev)
+        bsg_nvfp4_gemm(A, B, sfa, sfb, alpha, m_indices, out, M, N, K, G, stream)
     return out
+
+
+def moe_permute(expert_ids, G, stream=None):
+    """expert_ids int32 [T, top_k] (CUDA) -> (src_rows int32 [T*top_k], m_indices int32 [T*top_k],
+    dst_rows int32 [T, top_k], expert_offsets int32 [G+1]): the expert-grouped layout of the routing
+    entries (see bsg_moe_permute); the scratch is a torch allocation made here."""
+    import torch
+    _need(expert_ids, torch.int32, "expert_ids", 2)
+    T, top_k = expert_ids.shape
+    n = T * top_k
+    dev = _same_device((("expert_ids", expert_ids),), stream)
+    with torch.cuda.device(dev):
+        nbytes = bsg_moe_permute_workspace_size(T, top_k, G)
+        ws = torch.empty(max(16, nbytes), dtype=torch.uint8, device=dev)
+        src = torch.empty(n, dtype=torch.int32, device=dev)
+        mi = torch.empty(n, dtype=torch.int32, device=dev)
+        dst = torch.empty((T, top_k), dtype=torch.int32, device=dev)
+        off = torch.empty(G + 1, dtype=torch.int32, device=dev)
+        bsg_moe_permute(expert_ids, T, top_k, G, src, mi, dst, off, ws, ws.numel(), stream)
+    return src, mi, dst, off
 
 
 def quantize_fp8_rows(X, src_rows=None, stream=None):
@@ -316,9 +380,11 @@ def quantize_fp8_rows(X, src_rows=None, stream=None):
     if src_rows is not None:
         _need(src_rows, torch.int32, "src_rows", 1)
         M = src_rows.numel()
-    A = torch.zeros((M, K), dtype=torch.uint8, device=X.device)
-    s = torch.zeros((M, K // 128), dtype=torch.float32, device=X.device)
-    bsg_quantize_fp8_rows(X, src_rows, A, s, M_in, M, K, stream)
+    dev = _same_device((("X", X), ("src_rows", src_rows)), stream)
+    with torch.cuda.device(dev):
+        A = torch.zeros((M, K), dtype=torch.uint8, device=dev)
+        s = torch.zeros((M, K // 128), dtype=torch.float32, device=dev)
+        bsg_quantize_fp8_rows(X, src_rows, A, s, M_in, M, K, stream)
     return A, s
 
 
@@ -333,8 +399,10 @@ def quantize_nvfp4_rows(X, global_scale, src_rows=None, stream=None):
     if src_rows is not None:
         _need(src_rows, torch.int32, "src_rows", 1)
         M = src_rows.numel()
-    A = torch.zeros((M, K // 2), dtype=torch.uint8, device=X.device)
-    sf = torch.zeros((M, K // 16), dtype=torch.uint8, device=X.device)
-    bsg_quantize_nvfp4_rows(X, src_rows, global_scale, A, sf, M_in, M, K, stream)
+    dev = _same_device((("X", X), ("global_scale", global_scale), ("src_rows", src_rows)), stream)
+    with torch.cuda.device(dev):
+        A = torch.zeros((M, K // 2), dtype=torch.uint8, device=dev)
+        sf = torch.zeros((M, K // 16), dtype=torch.uint8, device=dev)
+        bsg_quantize_nvfp4_rows(X, src_rows, global_scale, A, sf, M_in, M, K, stream)
     return A, sf
 

@@ -22,6 +22,7 @@
 #include "bsg_chooser.h"
 #include "bsg_fp8.cuh"
 #include "bsg_fp8_swap.cuh"
+#include "bsg_moe.cuh"
 #include "bsg_nvfp4.cuh"
 
 #define BSG_VERSION_STRING "bsg 0.1.0 (sm_100a)"
@@ -54,6 +55,7 @@ struct DeviceState {
   bool fp8_attr = false;
   bool fp8_swap_attr = false;
   bool nvfp4_attr = false;
+  bool moe_attr = false;
   int fp8_pair_clusters = 0;
   int nvfp4_pair_clusters = 0;
 };
@@ -362,7 +364,8 @@ bsg_status fp8_launch(DeviceState* dev, const void* A, const void* B, const floa
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), static_cast<uint64_t>(G)};
     const uint64_t str[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N) * static_cast<uint64_t>(K)};
-    // B rows per CTA and stage: 256 (one SM, 256-column tile) or 64 (each CTA of an SM pair, 128-column tile)
+    // B rows per CTA and stage: 256 (one SM, 256-column tile) or 128 (each CTA of an SM pair, half of
+    // the pair's 256-column tile)
     const uint32_t box[3] = {128u, static_cast<uint32_t>(cg == 2 ? bsg::fp8::Cfg<2>::B_BOX_ROWS : bsg::fp8::Cfg<1>::B_BOX_ROWS), 1u};
     const bool oob[3] = {false, true, false};  // an N tail tile is zero-filled, columns masked
     if ((st = encode(&p.tmB, "B", B, 3, dims, str, box, oob, CU_TENSOR_MAP_SWIZZLE_128B)) != BSG_OK) return st;
@@ -561,9 +564,12 @@ bsg_status nvfp4_launch(DeviceState* dev, const void* A, const void* B, const vo
 }
 
 // Times `reps` launches of every tactic (after one warm-up launch each) with CUDA events on the
-// stream; returns the fastest tactic or a negative status.  `launch(t)` enqueues one call.
+// stream; returns the fastest tactic or a negative status.  `launch(t)` enqueues one call.  A tactic
+// whose launches gave up a bounded wait returned early and would look fastest: the device status
+// word is read (not cleared, so bsg_get_device_status still reports it) after each tactic, and a set
+// word ends the tuning with BSG_ERR_DEVICE_TIMEOUT and records nothing.
 template <typename Launch>
-int time_tactics(int kind, int reps, bsg_stream_t stream, Launch launch) {
+int time_tactics(DeviceState* dev, int kind, int reps, bsg_stream_t stream, Launch launch) {
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   cudaEvent_t ev[2];
   if (cudaEventCreate(&ev[0]) != cudaSuccess) return cuda_fail(cudaGetLastError(), "cudaEventCreate");
@@ -584,6 +590,18 @@ int time_tactics(int kind, int reps, bsg_stream_t stream, Launch launch) {
     if (st != BSG_OK) break;
     if (e != cudaSuccess) {
       st = cuda_fail(e, "timing a tactic");
+      break;
+    }
+    bsg::DeviceStatus hs = {0u, 0u};
+    e = cudaMemcpy(&hs, dev->status, sizeof(hs), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) {
+      st = cuda_fail(e, "reading the device status word");
+      break;
+    }
+    if (hs.word != 0u) {
+      st = fail(BSG_ERR_DEVICE_TIMEOUT,
+                "tactic %d (%s) gave up a bounded wait while being timed (status word 0x%08x); nothing recorded",
+                t, bsg_tactic_name(kind, t), hs.word);
       break;
     }
     float ms = 0.f;
@@ -632,7 +650,7 @@ int bsg_autotune_fp8(const void* A, const void* B, const float* a_scale, const f
   DeviceState* dev = nullptr;
   bsg_status st = fp8_check(A, B, a_scale, b_scale, m_indices, C, M, N, K, G, &dev);
   if (st != BSG_OK) return st;
-  const int best = time_tactics(0, reps, stream, [&](int t) {
+  const int best = time_tactics(dev, 0, reps, stream, [&](int t) {
     return fp8_launch(dev, A, B, a_scale, b_scale, m_indices, C, M, N, K, G, stream, t);
   });
   if (best >= 0) bsg_record_tuned(0, M, N, K, G, best);
@@ -647,7 +665,7 @@ int bsg_autotune_nvfp4(const void* A, const void* B, const void* sfa, const void
   DeviceState* dev = nullptr;
   bsg_status st = nvfp4_check(A, B, sfa, sfb, alpha, m_indices, C, M, N, K, G, &dev);
   if (st != BSG_OK) return st;
-  const int best = time_tactics(1, reps, stream, [&](int t) {
+  const int best = time_tactics(dev, 1, reps, stream, [&](int t) {
     return nvfp4_launch(dev, A, B, sfa, sfb, alpha, m_indices, C, M, N, K, G, stream, t);
   });
   if (best >= 0) bsg_record_tuned(1, M, N, K, G, best);
@@ -726,6 +744,124 @@ bsg_status bsg_quantize_nvfp4_rows(const void* X, const int32_t* src_rows, const
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launch of the nvfp4 quantisation kernel");
   return BSG_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Tiling of the MoE permutation: tiles of at least MIN_TILE entries (multiples of 32), at most
+// cap_ints / G of them, so that the scratch (tiles x G int32 counters) stays within cap_ints.
+struct MoePlan {
+  int tile = 0;
+  int tiles = 0;
+  size_t scratch_bytes = 0;
+};
+
+constexpr int64_t kMoeWorkspaceCapInts = 1ll << 22;  // 16 MiB of counters at most
+
+MoePlan moe_plan(int64_t n, int64_t G, int64_t cap_ints) {
+  MoePlan pl;
+  int64_t tiles = (n + bsg::moe::MIN_TILE - 1) / bsg::moe::MIN_TILE;
+  if (tiles < 1) tiles = 1;
+  if (tiles * G > cap_ints) tiles = cap_ints / G > 1 ? cap_ints / G : 1;
+  int64_t tile = (n + tiles - 1) / tiles;
+  tile = (tile + 31) / 32 * 32;
+  tiles = (n + tile - 1) / tile;
+  pl.tile = static_cast<int>(tile);
+  pl.tiles = static_cast<int>(tiles);
+  pl.scratch_bytes = static_cast<size_t>(tiles) * static_cast<size_t>(G) * sizeof(int32_t);
+  return pl;
+}
+
+bsg_status moe_check_sizes(int64_t T, int64_t top_k, int64_t G) {
+  if (T < 1 || top_k < 1 || top_k > 256)
+    return fail(BSG_ERR_UNSUPPORTED_SHAPE, "T = %lld and top_k = %lld must satisfy T >= 1, 1 <= top_k <= 256",
+                (long long)T, (long long)top_k);
+  if (T * top_k > (1ll << 24))
+    return fail(BSG_ERR_UNSUPPORTED_SHAPE, "T * top_k = %lld above 2^24 (the grouped GEMM's row limit)",
+                (long long)(T * top_k));
+  if (G < 1 || G > 4096) return fail(BSG_ERR_UNSUPPORTED_SHAPE, "G = %lld outside [1, 4096]", (long long)G);
+  return BSG_OK;
+}
+
+bsg_status moe_check(const int32_t* expert_ids, int64_t T, int64_t top_k, int64_t G, const int32_t* src_rows,
+                     const int32_t* m_indices, const int32_t* dst_rows, const int32_t* expert_offsets) {
+  bsg_status st = moe_check_sizes(T, top_k, G);
+  if (st != BSG_OK) return st;
+  if (!expert_ids || !src_rows || !m_indices || !dst_rows || !expert_offsets)
+    return fail(BSG_ERR_INVALID_ARG, "expert_ids, src_rows, m_indices, dst_rows and expert_offsets must be non-null");
+  if (!aligned(expert_ids, 4) || !aligned(src_rows, 4) || !aligned(m_indices, 4) || !aligned(dst_rows, 4) ||
+      !aligned(expert_offsets, 4))
+    return fail(BSG_ERR_ALIGNMENT, "the MoE permutation's int32 arrays must be 4-byte aligned");
+  return BSG_OK;
+}
+
+// The three kernels of the permutation on `stream`, with `scratch` (pl.scratch_bytes, 4-byte aligned).
+bsg_status moe_launch(DeviceState* dev, const int32_t* expert_ids, int64_t T, int64_t top_k, int64_t G,
+                      int32_t* src_rows, int32_t* m_indices, int32_t* dst_rows, int32_t* expert_offsets,
+                      int32_t* scratch, const MoePlan& pl, bsg_stream_t stream) {
+  cudaError_t e;
+  if (!dev->moe_attr) {
+    const int smem = bsg::moe::WARPS * 4096 * static_cast<int>(sizeof(int32_t));
+    e = cudaFuncSetAttribute(bsg::moe::bsg_moe_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(moe count kernel smem)");
+    e = cudaFuncSetAttribute(bsg::moe::bsg_moe_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(moe scatter kernel smem)");
+    dev->moe_attr = true;
+  }
+  bsg::moe::Params p;
+  memset(&p, 0, sizeof(p));
+  p.expert_ids = expert_ids;
+  p.src_rows = src_rows;
+  p.m_indices = m_indices;
+  p.dst_rows = dst_rows;
+  p.expert_offsets = expert_offsets;
+  p.scratch = scratch;
+  p.n = T * top_k;
+  p.top_k = static_cast<int>(top_k);
+  p.G = static_cast<int>(G);
+  p.tile = pl.tile;
+  p.tiles = pl.tiles;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const int blocks = (pl.tiles + bsg::moe::WARPS - 1) / bsg::moe::WARPS;
+  const size_t tile_smem = static_cast<size_t>(bsg::moe::WARPS) * static_cast<size_t>(G) * sizeof(int32_t);
+  bsg::moe::bsg_moe_count_kernel<<<blocks, bsg::moe::THREADS, tile_smem, cs>>>(p);
+  bsg::moe::bsg_moe_scan_kernel<<<1, bsg::moe::SCAN_THREADS, static_cast<size_t>(G) * sizeof(int32_t), cs>>>(p);
+  bsg::moe::bsg_moe_scatter_kernel<<<blocks, bsg::moe::THREADS, tile_smem, cs>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the MoE permutation kernels");
+  return BSG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+bsg_status bsg_moe_permute_workspace_size(int64_t T, int64_t top_k, int64_t G, size_t* bytes) {
+  g_last_error.clear();
+  if (!bytes) return fail(BSG_ERR_INVALID_ARG, "bytes must be non-null");
+  bsg_status st = moe_check_sizes(T, top_k, G);
+  if (st != BSG_OK) return st;
+  *bytes = moe_plan(T * top_k, G, kMoeWorkspaceCapInts).scratch_bytes;
+  return BSG_OK;
+}
+
+bsg_status bsg_moe_permute(const int32_t* expert_ids, int64_t T, int64_t top_k, int64_t G, int32_t* src_rows,
+                           int32_t* m_indices, int32_t* dst_rows, int32_t* expert_offsets, void* workspace,
+                           size_t workspace_bytes, bsg_stream_t stream) {
+  g_last_error.clear();
+  bsg_status st = moe_check(expert_ids, T, top_k, G, src_rows, m_indices, dst_rows, expert_offsets);
+  if (st != BSG_OK) return st;
+  const MoePlan pl = moe_plan(T * top_k, G, kMoeWorkspaceCapInts);
+  if (!workspace || workspace_bytes < pl.scratch_bytes)
+    return fail(BSG_ERR_INVALID_ARG, "workspace of %zu bytes is missing or smaller than the %zu bytes needed",
+                workspace_bytes, pl.scratch_bytes);
+  if (!aligned(workspace, 16)) return fail(BSG_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  DeviceState* dev = nullptr;
+  if ((st = device_state(&dev)) != BSG_OK) return st;
+  return moe_launch(dev, expert_ids, T, top_k, G, src_rows, m_indices, dst_rows, expert_offsets,
+                    static_cast<int32_t*>(workspace), pl, stream);
 }
 
 bsg_status bsg_get_device_status(bsg_stream_t stream) {

@@ -80,7 +80,7 @@ struct Cfg {
   static constexpr int B_BYTES = B_BOX_ROWS * BK;         // 32 KB (CG 1) / 16 KB (CG 2)
   static constexpr int STAGES = CG == 1 ? 4 : 6;          // 192 KB of ring either way
   static constexpr uint32_t STAGE_TX = CG * (A_BYTES + B_BYTES);  // bytes counted on the even CTA
-  static constexpr int EPI_COLS = BN / 4;                 // columns per epilogue warp: 64 / 32
+  static constexpr int EPI_COLS = BN / 4;                 // columns per epilogue warp: 64
   static constexpr int NB_TILE = BN / 128;                // 128-column scale blocks per tile
 };
 

@@ -222,3 +222,96 @@ def test_autotune_argument_errors(lib):
     assert ei.value.status == bsg.BSG_ERR_UNSUPPORTED_SHAPE
     bsg.bsg_autotune_clear()
 
+
+
+class _FakeDevice:
+    """Stand-in for a torch.device (the wrappers only compare devices)."""
+
+    def __init__(self, name):
+        self.name = name
+
+    def __eq__(self, other):
+        return isinstance(other, _FakeDevice) and other.name == self.name
+
+    def __repr__(self):
+        return self.name
+
+
+class _T:
+    def __init__(self, dev):
+        self.device = _FakeDevice(dev)
+
+
+def test_wrappers_reject_operands_on_different_devices():
+    ok = bsg._same_device((("A", _T("cuda:1")), ("B", _T("cuda:1")), ("m_indices", None)))
+    assert ok == _FakeDevice("cuda:1")
+    with pytest.raises(ValueError, match="out is on cuda:0"):
+        bsg._same_device((("A", _T("cuda:1")), ("B", _T("cuda:1")), ("out", _T("cuda:0"))))
+    with pytest.raises(ValueError, match="stream is on"):
+        bsg._same_device((("A", _T("cuda:1")),), stream=_T("cuda:0"))
+
+
+def test_nvfp4_wrapper_rejects_a_wrong_shaped_out_before_any_launch(monkeypatch):
+    import torch
+    calls = []
+    monkeypatch.setattr(bsg, "_need", lambda *a, **k: None)           # CPU tensors stand in for CUDA ones
+    monkeypatch.setattr(bsg, "bsg_nvfp4_gemm", lambda *a, **k: calls.append(a))
+    M, N, K, G = 256, 128, 512, 2
+    A = torch.zeros((M, K // 2), dtype=torch.uint8)
+    B = torch.zeros((G, N, K // 2), dtype=torch.uint8)
+    sfa = torch.zeros((M, K // 16), dtype=torch.uint8)
+    sfb = torch.zeros((G, N, K // 16), dtype=torch.uint8)
+    alpha = torch.ones(G)
+    idx = torch.zeros(M, dtype=torch.int32)
+    for bad in ((M - 1, N), (M, N - 8), (M, 2 * N)):
+        with pytest.raises(ValueError, match="out must be"):
+            bsg.nvfp4_gemm(A, B, sfa, sfb, alpha, idx, out=torch.zeros(bad, dtype=torch.bfloat16))
+    assert calls == []
+
+
+def test_fp8_wrapper_rejects_a_wrong_shaped_out_before_any_launch(monkeypatch):
+    import torch
+    calls = []
+    monkeypatch.setattr(bsg, "_need", lambda *a, **k: None)
+    monkeypatch.setattr(bsg, "bsg_fp8_grouped_gemm", lambda *a, **k: calls.append(a))
+    M, N, K, G = 256, 128, 512, 2
+    A = torch.zeros((M, K), dtype=torch.uint8)
+    B = torch.zeros((G, N, K), dtype=torch.uint8)
+    with pytest.raises(ValueError, match="out must be"):
+        bsg.fp8_grouped_gemm(A, B, torch.ones(M, K // 128), torch.ones(G, 1, K // 128),
+                             torch.zeros(M, dtype=torch.int32), out=torch.zeros((M, N + 8), dtype=torch.bfloat16))
+    assert calls == []
+
+
+def test_moe_permute_workspace_size(lib):
+    # tiles of at least 256 entries (multiples of 32), one row of G int32 counters per tile
+    assert bsg.bsg_moe_permute_workspace_size(8192, 8, 8) == 256 * 8 * 4
+    assert bsg.bsg_moe_permute_workspace_size(1, 1, 1) == 4
+    assert bsg.bsg_moe_permute_workspace_size(100, 3, 64) == 2 * 64 * 4
+    # capped at 2^22 counters (16 MiB): G = 4096 allows 1024 tiles
+    assert bsg.bsg_moe_permute_workspace_size(1 << 21, 8, 4096) == 1024 * 4096 * 4
+    for T, k, G, needle in ((0, 1, 4, "T = 0"), (4, 0, 4, "top_k = 0"), (4, 300, 4, "256"),
+                            (1 << 22, 8, 4, "2^24"), (4, 2, 0, "G = 0"), (4, 2, 5000, "4096")):
+        with pytest.raises(bsg.BsgError) as ei:
+            bsg.bsg_moe_permute_workspace_size(T, k, G)
+        assert ei.value.status == bsg.BSG_ERR_UNSUPPORTED_SHAPE and needle in str(ei.value)
+
+
+@pytest.mark.parametrize("kw,status,needle", [
+    (dict(expert_ids=0), bsg.BSG_ERR_INVALID_ARG, "non-null"),
+    (dict(dst_rows=0), bsg.BSG_ERR_INVALID_ARG, "non-null"),
+    (dict(workspace=0), bsg.BSG_ERR_INVALID_ARG, "workspace"),
+    (dict(workspace_bytes=4), bsg.BSG_ERR_INVALID_ARG, "smaller"),
+    (dict(workspace=FAKE + 4), bsg.BSG_ERR_ALIGNMENT, "16-byte"),
+    (dict(src_rows=FAKE + 2), bsg.BSG_ERR_ALIGNMENT, "4-byte"),
+    (dict(T=1 << 22, top_k=8), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "2^24"),
+    (dict(G=0), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "G = 0"),
+])
+def test_moe_permute_argument_errors(lib, kw, status, needle):
+    a = dict(expert_ids=FAKE, T=512, top_k=2, G=8, src_rows=FAKE, m_indices=FAKE, dst_rows=FAKE,
+             expert_offsets=FAKE, workspace=FAKE, workspace_bytes=1 << 20)
+    a.update(kw)
+    with pytest.raises(bsg.BsgError) as ei:
+        bsg.bsg_moe_permute(**a, stream=0)
+    assert ei.value.status == status
+    assert needle in str(ei.value)

@@ -217,6 +217,34 @@ def test_fp8_bounded_wait_reports_timeout_and_context_survives():
     compare(out, oracle_rows(w), routed_mask(w))
 
 
+def test_fp8_autotune_under_expired_waits_records_nothing():
+    """Autotune while every bounded wait expires (host-side fault injection, 50 ms limit): the
+    launches return early and would look fastest, so the tuning must report BSG_ERR_DEVICE_TIMEOUT
+    and record no tactic; the context stays usable."""
+    w = W.config(0)
+    d = DevWorkload(w)
+    C = sentinel_out(w.M, w.N)
+    bsg.bsg_autotune_clear()
+    prev = bsg.bsg_set_wait_timeout_ns(50_000_000)
+    try:
+        bsg.bsg_debug_set_fault(1)
+        with pytest.raises(bsg.BsgError) as ei:
+            bsg.bsg_autotune_fp8(d.A, d.B, d.a_scale, d.b_scale, d.m_indices, C, w.M, w.N, w.K, w.G, reps=1)
+        assert ei.value.status == bsg.BSG_ERR_DEVICE_TIMEOUT
+    finally:
+        bsg.bsg_debug_set_fault(0)
+        bsg.bsg_set_wait_timeout_ns(prev)
+    with pytest.raises(bsg.BsgError):
+        bsg.bsg_get_device_status()                     # the word stayed set for the caller to see
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    forced_free = bsg.bsg_choose_tactic(0, w.M, w.N, w.K, w.G, sms)
+    bsg.bsg_autotune_clear()
+    assert forced_free == bsg.bsg_choose_tactic(0, w.M, w.N, w.K, w.G, sms)   # nothing was recorded
+    out = bits(d.run())
+    bsg.bsg_get_device_status()
+    compare(out, oracle_rows(w), routed_mask(w))
+
+
 def test_fp8_torch_wrapper():
     w = W.config(0)
     d = DevWorkload(w)
