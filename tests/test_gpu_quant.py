@@ -172,3 +172,39 @@ def test_tiny_scales_and_signed_zeros():
         A4_ref, sf_ref = oracle.quant_nvfp4_rows(rows, gs)
         assert np.array_equal(sf.cpu().numpy(), sf_ref), f"gs {gs!r}"
         assert np.array_equal(A4.cpu().numpy(), A4_ref), f"gs {gs!r}"
+
+
+def test_every_bf16_block_maximum():
+    """Blocks whose maximum takes every positive bf16 value (the scale divisions amax / 448 and
+    amax / 6 are computed without a division instruction): scales and codes bit-exact."""
+    rng = np.random.default_rng(50)
+    amax_bits = np.arange(0x0001, 0x7F80, dtype=np.uint16)
+    # FP8: 128-element blocks, 128 blocks per row
+    n = ((amax_bits.size + 127) // 128) * 128
+    am = np.resize(amax_bits, n)
+    blocks = (rng.uniform(-1, 1, (n, 128)).astype(np.float32)
+              * (am.astype(np.uint32) << 16).view(np.float32)[:, None]).astype(np.float32)
+    bits16 = (blocks.view(np.uint32) >> 16).astype(np.uint16)
+    bits16[:, 0] = am
+    rows = bits16.reshape(-1, 128 * 128)
+    xt = torch.from_numpy(rows.view(np.int16).copy()).view(torch.bfloat16)
+    A, s = bsg.quantize_fp8_rows(xt.cuda())
+    torch.cuda.synchronize()
+    A_ref, s_ref = oracle.quant_fp8_rows(rows)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(A.cpu().numpy(), A_ref)
+    # NVFP4: 16-element blocks, 1024 blocks per row, two global scales
+    n = ((amax_bits.size + 1023) // 1024) * 1024
+    am = np.resize(amax_bits, n)
+    blocks = (rng.uniform(-1, 1, (n, 16)).astype(np.float32)
+              * (am.astype(np.uint32) << 16).view(np.float32)[:, None]).astype(np.float32)
+    bits16 = (blocks.view(np.uint32) >> 16).astype(np.uint16)
+    bits16[:, 0] = am
+    rows = bits16.reshape(-1, 16 * 1024)
+    xt = torch.from_numpy(rows.view(np.int16).copy()).view(torch.bfloat16)
+    for gs in (np.float32(1.0 / 2688.0), np.float32(3.1e-7), np.float32(1.7e-30)):
+        A4, sf = bsg.quantize_nvfp4_rows(xt.cuda(), torch.tensor([gs], dtype=torch.float32, device="cuda"))
+        torch.cuda.synchronize()
+        A4_ref, sf_ref = oracle.quant_nvfp4_rows(rows, gs)
+        assert np.array_equal(sf.cpu().numpy(), sf_ref), f"gs {gs!r}"
+        assert np.array_equal(A4.cpu().numpy(), A4_ref), f"gs {gs!r}"
