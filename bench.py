@@ -6,15 +6,16 @@
 
 One step = one launch of the whole hot path (window scheduling, TMA loads, scale handling, tcgen05
 MMAs, BF16 epilogue -- all inside one kernel) over one batch of synthetic input.  The headline
-workload is the FP8 grouped MoE prefill (G=8, M=8192, N=4096, K=7168); `--config` picks another of
-the five workloads.  The timed region is K back-to-back launches bracketed by a barrier and a device
+workload is the largest of the five, the NVFP4 grouped GEMM (G=8, M_g=8192, N=K=8192); `--config`
+picks another.  The timed region is K back-to-back launches bracketed by a barrier and a device
 synchronisation, timed with CUDA events on the launching stream, max over ranks.  Inputs are larger
 than the 126 MB L2 for the headline workload (stated in the JSON `config`); smaller workloads flush
 L2 between launches outside the per-launch events.
 
 Rank 0 prints ONE JSON line (metric, value = whole-job TFLOPS, roofline of the kernel, the oracle's
 CPU throughput on a bounded sample, the end-to-end number through host buffers, clocks sampled
-during the timed region).  `--impl reference` times the fp64 CPU oracle on the same workload instead
+during the timed region); on one GPU the line's `also` holds the same fields for each of the other
+four workloads, and the activation quantisers' HBM throughput.  `--impl reference` times the fp64 CPU oracle on the same workload instead
 (rank 0 only).  Under torchrun each rank runs its own copy of the workload on its own GPU (weak
 scaling, no data-path collective: the op needs no exchange step).
 """
@@ -34,6 +35,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "grouped block-scaled GEMM TFLOPS (FP8 & NVFP4) + % of B200 roofline"
+# The headline workload: the largest of the five (NVFP4 grouped, G=8, M_g=8192, N=K=8192, 8.8 TFLOP);
+# the metric names no single workload, so the largest one is the headline and the others are reported
+# beside it with the same fields.
+HEADLINE_CONFIG = 3
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # nominal dense ratios to bf16 (2.25 PF): fp8 4.5 PF, fp4 9 PF
@@ -46,7 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["bsg", "reference"], default="bsg")
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--config", type=int, default=HEADLINE_CONFIG)
     ap.add_argument("--no-also", action="store_true", help="skip the other workloads' kernel numbers")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     ap.add_argument("--e2e-steps", type=int, default=20)
@@ -113,8 +118,15 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 100 ms while running."""
+    """SM clock, its maximum and the throttle reasons, sampled while the timed region runs.
 
+    NVML (read-only queries) is polled every millisecond from a thread, so even a timed region of a
+    few milliseconds gets samples; without NVML, nvidia-smi is polled every 100 ms."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
@@ -122,10 +134,52 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
         self.thread = None
+        self.stop_flag = threading.Event()
+        self.samples = []          # (sm_mhz, max_mhz, set of active reason names)
+        self.source = None
+        self.nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+            self.masks = [(name, getattr(pynvml, attr, 0)) for name, attr in self.REASONS]
+        except Exception:
+            self.nvml = None
+
+    def _poll_nvml(self):
+        nv = self.nvml
+        while not self.stop_flag.is_set():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+                bits = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle))
+                self.samples.append((sm, self.max_mhz, {n for n, m in self.masks if m and bits & m}))
+            except Exception:
+                pass
+            time.sleep(0.001)
+
+    def _read_smi(self):
+        names = [n for n, _ in self.REASONS]
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.strip().split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm, mx = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            self.samples.append((sm, mx, {n for n, v in zip(names, parts[4:8]) if v.lower() == "active"}))
 
     def start(self):
+        self.samples = []
+        self.stop_flag.clear()
+        if self.nvml is not None:
+            self.source = "nvml, 1 ms"
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.thread.start()
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
@@ -133,41 +187,28 @@ class ClockSampler:
         except (OSError, FileNotFoundError):
             self.proc = None
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.source = "nvidia-smi, 100 ms"
+        self.thread = threading.Thread(target=self._read_smi, daemon=True)
         self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
+        self.stop_flag.set()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.proc = None
         if self.thread:
             self.thread.join(timeout=2)
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set()
+        for _, _, r in self.samples:
+            reasons |= r
+        return {"sm_mhz": statistics.median(x[0] for x in self.samples), "sm_max_mhz": self.samples[-1][1],
+                "reasons": sorted(reasons), "samples": len(self.samples), "source": self.source}
 
 
 def visible_gpu_index(local_rank):
@@ -192,17 +233,22 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload_name):
-    """DRAM bytes per launch from a committed ncu capture, if taken on the current kernel sources."""
+def recorded_profile(workload_name):
+    """The committed ncu figures of one workload's kernel (profiles/traffic.json): DRAM bytes per
+    launch and tensor-pipe activity, if taken on the current kernel sources; else {}."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
-        return None
+        return {}
     with open(p) as f:
         d = json.load(f)
     e = d.get(workload_name)
     if not e or e.get("source_hash") != kernel_source_hash():
-        return None
-    return e.get("bytes_per_launch")
+        return {}
+    return e
+
+
+def recorded_traffic(workload_name):
+    return recorded_profile(workload_name).get("bytes_per_launch")
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -250,9 +296,10 @@ def torch_sm_count():
     return torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
 
 
-def time_kernel(runner, steps, warmup, flush=None):
+def time_kernel(runner, steps, warmup, flush=None, sampler=None):
     """K back-to-back launches between synchronisations; returns (total seconds, mean per-launch
-    seconds from per-launch event pairs on the launching stream)."""
+    seconds from per-launch event pairs on the launching stream, clocks sampled during the timed
+    region or None)."""
     import torch
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
@@ -265,6 +312,8 @@ def time_kernel(runner, steps, warmup, flush=None):
     t1 = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.start()
     t0.record(stream)
     for i in range(steps):
         if flush is not None:
@@ -274,11 +323,12 @@ def time_kernel(runner, steps, warmup, flush=None):
         ends[i].record(stream)
     t1.record(stream)
     torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler is not None else None
     barrier()
     runner.bsg.bsg_get_device_status()
     total = t0.elapsed_time(t1) / 1e3
     per = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / steps / 1e3
-    return total, per
+    return total, per, clocks
 
 
 def time_e2e(runner, steps):
@@ -354,8 +404,11 @@ def roofline(w, per_launch_s, peaks, peak_src, sustained=False):
     return {"bound": "tensor", "achieved": round(ach, 1), "peak": round(tensor_peak, 1), "unit": "TFLOP/s",
             "frac": round(ach / tensor_peak, 4), "frac_of_sustained_peak": round(ach / sustained_peak, 4),
             "traffic": traffic, "algorithmic_bytes": nbytes,
-            "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} x {DTYPE_RATIO[w.kind]:g} "
-                           f"({w.kind} : bf16 nominal dense ratio)"}
+            "tensor_pipe_active_pct_ncu": recorded_profile(w.name).get("tensor_pipe_pct"),
+            "peak_source": f"derived: {peak_src} bf16 {'sustained' if sustained else 'burst'} "
+                           f"{peaks['bf16_tflops_sustained' if sustained else 'bf16_tflops']} TFLOP/s x "
+                           f"{DTYPE_RATIO[w.kind]:g} ({w.kind} : bf16 nominal dense ratio); no {w.kind} "
+                           f"peak is measured on this pool"}
 
 
 def time_quantiser(kind, M, K, peaks, steps=50, warmup=5):
@@ -403,6 +456,40 @@ def time_quantiser(kind, M, K, peaks, steps=50, warmup=5):
             "l2": "flushed" if flush else "inputs > L2"}
 
 
+def time_moe_permute(T, top_k, G, peaks, steps=50, warmup=5):
+    """The MoE expand permutation (three kernel launches: per-tile counts, scan, stable scatter) on a
+    Zipf-skewed routing of T tokens x top_k choices over G experts.  Integer work bound by the
+    latency of its dependent steps; reported with the HBM bytes it must move."""
+    import torch
+    import nvfp4_grouped_gemm_indices_b200 as bsg
+    g = torch.Generator(device="cuda").manual_seed(T * 131 + G)
+    ranks = torch.arange(1, G + 1, dtype=torch.float64, device="cuda") ** -1.2
+    ids = torch.multinomial((ranks / ranks.sum()).float(), T * top_k, replacement=True, generator=g)
+    ids = ids.to(torch.int32).view(T, top_k)
+    n = T * top_k
+    ws = torch.empty(max(16, bsg.bsg_moe_permute_workspace_size(T, top_k, G)), dtype=torch.uint8, device="cuda")
+    outs = [torch.empty(n, dtype=torch.int32, device="cuda"), torch.empty(n, dtype=torch.int32, device="cuda"),
+            torch.empty((T, top_k), dtype=torch.int32, device="cuda"),
+            torch.empty(G + 1, dtype=torch.int32, device="cuda")]
+    stream = torch.cuda.current_stream()
+    launch = lambda: bsg.bsg_moe_permute(ids, T, top_k, G, *outs, ws, ws.numel(), stream.cuda_stream)
+    for _ in range(warmup):
+        launch()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        launch()
+    b.record(stream)
+    b.synchronize()
+    per = a.elapsed_time(b) / 1e3 / steps
+    nbytes = 2 * 4 * n + 3 * 4 * n + 4 * (G + 1)      # ids read twice; src, m_indices, dst written
+    return {"us_per_launch": round(per * 1e6, 2), "kernel_launches": 3,
+            "hbm_bytes": nbytes, "achieved_gbs": round(nbytes / per / 1e9, 1),
+            "note": "latency-bound integer work; back-to-back launches, inputs L2-resident"}
+
+
 def cpu_baseline(w, seconds):
     """The oracle as it stands, on the host's cores, over a bounded sample of the workload's rows
     (all N columns each).  Returns (TFLOPS, cores, sample description)."""
@@ -440,14 +527,53 @@ def run_oracle(w, rows, n_cols=None):
                         w.G, rows=rows)
 
 
-def config_desc(w, cfg, flush):
+def needs_flush(w):
+    """Inputs smaller than twice the L2 are flushed out of it between timed launches."""
+    return (w.A.nbytes + w.B.nbytes) < 2 * L2_BYTES
+
+
+def config_desc(w, cfg):
+    """The workload, identically for both arms (sizes only; nothing that depends on the GPU)."""
     d = {"workload": w.name, "config_index": cfg, "kind": w.kind, "M": w.M, "N": w.N, "K": w.K, "G": w.G,
          "routed_rows": w.routed_rows, "active_experts": len(w.active_experts()),
          "input_bytes": int(w.A.nbytes + w.B.nbytes + (w.m_indices.nbytes if w.m_indices is not None else 0)),
          "parallelism": "replicas (one independent batch per GPU, no collective)"}
-    d["l2"] = ("L2 flushed (2x126 MB written, then 2x126 MB read: cold and clean) between launches, outside the per-launch events" if flush
+    d["l2"] = ("L2 flushed (2x126 MB written, then 2x126 MB read: cold and clean) between launches, outside the "
+               "per-launch events" if needs_flush(w)
                else f"inputs {d['input_bytes'] / 1e6:.0f} MB > 126 MB L2, no flush")
     return d
+
+
+def dtype_desc(w):
+    return ("e4m3xe4m3->f32 (fp32 per-128 scales), bf16 out" if w.kind == "fp8"
+            else "e2m1xe2m1 (ue4m3 per-16 scales)->f32, bf16 out")
+
+
+def measure(w, cfg, steps, warmup, e2e_steps, cpu_seconds, peaks, peak_src, sampler, ws, rank):
+    """Kernel time (device-resident inputs), end-to-end time through host buffers, and (rank 0 of a
+    single-GPU run) the oracle's CPU throughput on a bounded sample, for one workload."""
+    r = Runner(w)
+    flush = make_flush() if needs_flush(w) else None
+    total, per, clocks = time_kernel(r, steps, warmup, flush, sampler)
+    if flush is not None:
+        total = per * steps                 # the flushes between launches are not the kernel's time
+    total = reduce_max(total, device="cuda")
+    per = reduce_max(per, device="cuda")
+    e2e_s, h2d, d2h = time_e2e(r, e2e_steps)
+    e2e_s = reduce_max(e2e_s, device="cuda")
+    out = {
+        "value": round(job_value(w.flops, total / steps, ws), 2), "ms_per_step": round(total / steps * 1e3, 5),
+        "us_per_launch": round(per * 1e6, 2), "tactic": r.tactic(), "config": config_desc(w, cfg),
+        "roofline": roofline(w, per, peaks, peak_src), "clocks": clocks, "gpu_launches": steps,
+        "e2e": {"value": round(job_value(w.flops, e2e_s, ws), 3), "unit": "TFLOPS", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
+                "note": "all operands copied host->device from pinned memory and C copied back, every step"},
+    }
+    del r
+    if ws == 1 and rank == 0:
+        tf, cores, sample = cpu_baseline(w, cpu_seconds)
+        out["cpu_baseline"] = {"value": tf, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample}
+    return out
 
 
 def run_bsg(args):
@@ -463,61 +589,36 @@ def run_bsg(args):
     sampler = ClockSampler(visible_gpu_index(local))
     from nvfp4_grouped_gemm_indices_b200 import workloads as W
     w = W.config(args.config)
-    r = Runner(w)
-    flush = make_flush() if (w.A.nbytes + w.B.nbytes) < 2 * L2_BYTES else None
-    sampler.start()
-    total, per = time_kernel(r, args.steps, args.warmup, flush)
-    clocks = sampler.stop()
-    if flush is not None:
-        total = per * args.steps
-    total = reduce_max(total, device="cuda")
-    per = reduce_max(per, device="cuda")
-    ms_per_step = total / args.steps * 1e3
-    value = job_value(w.flops, total / args.steps, ws)
-
-    e2e_s, h2d, d2h = time_e2e(r, args.e2e_steps)
-    e2e_s = reduce_max(e2e_s, device="cuda")
-    e2e_value = job_value(w.flops, e2e_s, ws)
-
+    m = measure(w, args.config, args.steps, args.warmup, args.e2e_steps, args.cpu_seconds, peaks, peak_src,
+                sampler, ws, rank)
     line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3xe4m3->f32 (fp32 per-128 scales), bf16 out" if w.kind == "fp8"
-        else "e2m1xe2m1 (ue4m3 per-16 scales)->f32, bf16 out",
+        "metric": METRIC, "value": m["value"], "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype_desc(w),
         "data": "synthetic (seeded; quantised N(0,1) activations, N(0,0.02) / N(0,1) weights)",
-        "config": dict(config_desc(w, args.config, flush), tactic=r.tactic()),
-        "roofline": roofline(w, per, peaks, peak_src),
-        "gpu_launches": args.steps,
-        "clocks": clocks,
-        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS", "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps,
-                "note": "all operands copied host->device from pinned memory and C copied back, every step"},
+        "config": m["config"], "tactic": m["tactic"], "roofline": m["roofline"],
+        "gpu_launches": m["gpu_launches"], "clocks": m["clocks"], "e2e": m["e2e"],
     }
-    if ws == 1 and rank == 0:
-        tf, cores, sample = cpu_baseline(w, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": tf, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample}
-        if not args.no_also:
-            also = {}
-            for cfg in (0, 2, 3, 4):
-                if cfg == args.config:
-                    continue
-                del r
-                torch.cuda.empty_cache()
-                wc = W.config(cfg)
-                r = Runner(wc)
-                fl = make_flush() if (wc.A.nbytes + wc.B.nbytes) < 2 * L2_BYTES else None
-                steps = max(20, min(args.steps, 200))
-                tot, pl = time_kernel(r, steps, max(3, args.warmup // 4), fl)
-                rf = roofline(wc, pl, peaks, peak_src)
-                also[wc.name] = {"tactic": r.tactic(), "tflops": round(wc.flops / pl / 1e12, 2),
-                                 "us_per_launch": round(pl * 1e6, 2),
-                                 "roofline": rf, "l2": "flushed" if fl else "inputs > L2"}
-            del r
+    if "cpu_baseline" in m:
+        line["cpu_baseline"] = m["cpu_baseline"]
+    del w
+    torch.cuda.empty_cache()
+    if ws == 1 and rank == 0 and not args.no_also:
+        also = {}
+        for cfg in range(5):
+            if cfg == args.config:
+                continue
+            wc = W.config(cfg)
+            also[wc.name] = measure(wc, cfg, max(20, min(args.steps, 200)), max(3, args.warmup),
+                                    min(args.e2e_steps, 10), max(4.0, args.cpu_seconds / 3), peaks, peak_src,
+                                    sampler, ws, rank)
+            del wc
             torch.cuda.empty_cache()
-            also["quant_fp8_rows_gather_m8192_k7168"] = time_quantiser("fp8", 8192, 7168, peaks)
-            also["quant_nvfp4_rows_gather_m65536_k8192"] = time_quantiser("nvfp4", 65536, 8192, peaks)
-            line["also"] = also
+        also["quant_fp8_rows_gather_m8192_k7168"] = time_quantiser("fp8", 8192, 7168, peaks)
+        also["quant_nvfp4_rows_gather_m65536_k8192"] = time_quantiser("nvfp4", 65536, 8192, peaks)
+        also["moe_permute_t8192_k8_g64"] = time_moe_permute(8192, 8, 64, peaks)
+        also["moe_permute_t64_k8_g64"] = time_moe_permute(64, 8, 64, peaks)
+        line["also"] = also
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -557,8 +658,9 @@ def run_reference(args):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (decoded operands)", "data": "synthetic",
-        "config": {"workload": w.name, "config_index": args.config, "M": w.M, "N": w.N, "K": w.K, "G": w.G},
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (decoded operands; " + dtype_desc(w) + " inputs)",
+        "data": "synthetic (seeded; quantised N(0,1) activations, N(0,0.02) / N(0,1) weights)",
+        "config": config_desc(w, args.config),
         "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -610,7 +712,7 @@ def run_sweep(args):
         times = {}
         for t in range(bsg.bsg_num_tactics(kind)):
             bsg.bsg_set_tactic(kind, t)
-            _, per = time_kernel(r, max(10, min(args.steps, 100)), 3, flush)
+            _, per, _ = time_kernel(r, max(10, min(args.steps, 100)), 3, flush)
             times[bsg.bsg_tactic_name(kind, t)] = per
         bsg.bsg_set_tactic(kind, -1)
         pick = bsg.bsg_tactic_name(kind, bsg.bsg_choose_tactic(kind, w.M, w.N, w.K, w.G, sms))
