@@ -150,6 +150,30 @@ bsg_status bsg_moe_permute(const int32_t* expert_ids, int64_t T, int64_t top_k, 
                            int32_t* m_indices, int32_t* dst_rows, int32_t* expert_offsets, void* workspace,
                            size_t workspace_bytes, bsg_stream_t stream);
 
+/*
+ * bsg_moe_permute without a workspace argument, for callers that cannot allocate device memory:
+ * a plugin whose host application owns every device allocation and hands it no allocator, a
+ * serving loop that must not call cudaMalloc / cudaFree (they can synchronise the whole device and
+ * stall the other streams), or a process that has to keep its device footprint fixed after start-up.
+ * (This entry point has no counterpart in the pages the library follows; it is the same permutation
+ * as bsg_moe_permute, with identical results.)
+ *
+ * The scratch is a fixed 2 MiB array that the library's device image carries on every GPU that loads
+ * it, for as long as the process lives.  Limit: the sizes (T, top_k, G) whose
+ * bsg_moe_permute_workspace_size() is at most 2 MiB -- for example T * top_k up to 2^21 entries with
+ * G = 64, 2^19 with G = 256, 2^14 with G = 4096; larger sizes return BSG_ERR_UNSUPPORTED_SHAPE with a
+ * message and launch nothing.  The first call on a device also looks up that device's copy of the
+ * array (with the device current), so make that first call before capturing any stream.
+ * Every call on a device shares the one array and leaves its last contents behind; the kernels
+ * overwrite every counter before they read it, so nothing needs clearing between calls, but calls
+ * that overlap on the GPU (different streams, no ordering between them) race on the array and give
+ * undefined results.  Nothing is allocated or freed, by this call or by anything it calls.
+ * Arguments, outputs, contract and asynchrony otherwise as for bsg_moe_permute.
+ */
+bsg_status bsg_moe_permute_noalloc(const int32_t* expert_ids, int64_t T, int64_t top_k, int64_t G,
+                                   int32_t* src_rows, int32_t* m_indices, int32_t* dst_rows,
+                                   int32_t* expert_offsets, bsg_stream_t stream);
+
 /* Description of the last failure on the calling thread ("" if none).  The string stays valid until
  * the next bsg_* call on the same thread. */
 const char* bsg_last_error(void);

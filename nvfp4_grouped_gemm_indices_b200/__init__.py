@@ -49,7 +49,7 @@ EXPORTED = [
     "bsg_set_wait_timeout_ns", "bsg_num_tactics", "bsg_tactic_name", "bsg_choose_tactic",
     "bsg_tactic_score", "bsg_set_tactic", "bsg_set_max_ctas", "bsg_debug_set_fault", "bsg_version",
     "bsg_quantize_fp8_rows", "bsg_quantize_nvfp4_rows", "bsg_autotune_fp8", "bsg_autotune_nvfp4",
-    "bsg_autotune_clear", "bsg_moe_permute_workspace_size", "bsg_moe_permute",
+    "bsg_autotune_clear", "bsg_moe_permute_workspace_size", "bsg_moe_permute", "bsg_moe_permute_noalloc",
 ]
 
 
@@ -112,6 +112,8 @@ def load(path: Optional[str] = None):
     L.bsg_moe_permute_workspace_size.argtypes = [i64, i64, i64, ctypes.POINTER(ctypes.c_size_t)]
     L.bsg_moe_permute.restype = i32
     L.bsg_moe_permute.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    L.bsg_moe_permute_noalloc.restype = i32
+    L.bsg_moe_permute_noalloc.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp]
     if path is None:
         _lib = L
     return L
@@ -178,6 +180,13 @@ def bsg_moe_permute(expert_ids, T, top_k, G, src_rows, m_indices, dst_rows, expe
     _check(load().bsg_moe_permute(_ptr(expert_ids), int(T), int(top_k), int(G), _ptr(src_rows), _ptr(m_indices),
                                   _ptr(dst_rows), _ptr(expert_offsets), _ptr(workspace), int(workspace_bytes),
                                   _stream(stream)))
+
+
+def bsg_moe_permute_noalloc(expert_ids, T, top_k, G, src_rows, m_indices, dst_rows, expert_offsets, stream=None):
+    """bsg_moe_permute for callers that cannot allocate device memory: the scratch is a fixed 2 MiB
+    array inside the library (see include/bsg.h for the size limit and the sharing rules)."""
+    _check(load().bsg_moe_permute_noalloc(_ptr(expert_ids), int(T), int(top_k), int(G), _ptr(src_rows),
+                                          _ptr(m_indices), _ptr(dst_rows), _ptr(expert_offsets), _stream(stream)))
 
 
 def bsg_autotune_fp8(A, B, a_scale, b_scale, m_indices, C, M, N, K, G, reps=20, stream=None) -> int:

@@ -864,6 +864,60 @@ bsg_status bsg_moe_permute(const int32_t* expert_ids, int64_t T, int64_t top_k, 
                     static_cast<int32_t*>(workspace), pl, stream);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Scratch of bsg_moe_permute_noalloc: one array in the library's device image (every GPU that loads
+// the library holds it until the process exits), shared by every call on that GPU.  Host code sees
+// only a host-side stand-in under this name, so the device address is looked up once per device.
+constexpr size_t kMoeStaticScratchBytes = 2u << 20;   // 2 MiB = 524288 int32 counters
+static __device__ __align__(256) int32_t g_moe_static_scratch[kMoeStaticScratchBytes / sizeof(int32_t)];
+
+int32_t* g_moe_static_addr[kMaxDevices] = {};
+
+// The device address of the static scratch on the current device (looked up on the first call for
+// that device, with that device current).
+bsg_status moe_static_scratch(int32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(BSG_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_moe_static_addr[dev]) {
+    void* addr = nullptr;
+    e = cudaGetSymbolAddress(&addr, g_moe_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(MoE permutation scratch)");
+    g_moe_static_addr[dev] = static_cast<int32_t*>(addr);
+  }
+  *out = g_moe_static_addr[dev];
+  return BSG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+bsg_status bsg_moe_permute_noalloc(const int32_t* expert_ids, int64_t T, int64_t top_k, int64_t G,
+                                   int32_t* src_rows, int32_t* m_indices, int32_t* dst_rows,
+                                   int32_t* expert_offsets, bsg_stream_t stream) {
+  g_last_error.clear();
+  bsg_status st = moe_check(expert_ids, T, top_k, G, src_rows, m_indices, dst_rows, expert_offsets);
+  if (st != BSG_OK) return st;
+  const MoePlan pl = moe_plan(T * top_k, G, kMoeWorkspaceCapInts);
+  if (pl.scratch_bytes > kMoeStaticScratchBytes)
+    return fail(BSG_ERR_UNSUPPORTED_SHAPE,
+                "T = %lld, top_k = %lld, G = %lld need %zu bytes of scratch, more than the %zu bytes this "
+                "allocation-free entry point holds; call bsg_moe_permute with a workspace instead",
+                (long long)T, (long long)top_k, (long long)G, pl.scratch_bytes, kMoeStaticScratchBytes);
+  DeviceState* dev = nullptr;
+  if ((st = device_state(&dev)) != BSG_OK) return st;
+  int32_t* scratch = nullptr;
+  if ((st = moe_static_scratch(&scratch)) != BSG_OK) return st;
+  return moe_launch(dev, expert_ids, T, top_k, G, src_rows, m_indices, dst_rows, expert_offsets, scratch, pl,
+                    stream);
+}
+
 bsg_status bsg_get_device_status(bsg_stream_t stream) {
   g_last_error.clear();
   DeviceState* dev = nullptr;
