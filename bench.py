@@ -685,6 +685,10 @@ def sweep_shapes():
     for (M, N, K, G) in [(2048, 4096, 7168, 8), (4096, 2048, 4096, 16), (1024, 7168, 2048, 32), (16384, 4096, 4096, 4)]:
         idx = W.counts_to_indices(rng.multinomial(M, [1.0 / G] * G))
         out.append(W.make_fp8(M, N, K, G, idx, seed=M + N, name=f"fp8_sweep_g{G}_m{M}_n{N}_k{K}"))
+    # the FP8 page's two benchmark shapes (small launches)
+    for (M, N, K, G) in [(65, 128, 128, 2), (777, 256, 512, 8)]:
+        counts = [M // G + (1 if i < M % G else 0) for i in range(G)]
+        out.append(W.make_fp8(M, N, K, G, W.counts_to_indices(counts), seed=M, name=f"fp8_page_g{G}_m{M}_n{N}_k{K}"))
     # few rows per expert (decode): where the operand-swapped tiles take over from the row tiles
     idx = W.routing_zipf(96, 32, rng)
     out.append(W.make_fp8(96, 2048, 4096, 32, idx, seed=96, name="fp8_sweep_zipf_g32_m96_n2048_k4096"))

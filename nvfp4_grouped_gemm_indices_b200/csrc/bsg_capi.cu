@@ -54,6 +54,7 @@ struct DeviceState {
   bsg::DeviceStatus* status = nullptr;
   bool fp8_attr = false;
   bool fp8_swap_attr = false;
+  bool fp8_n64_attr = false;
   bool nvfp4_attr = false;
   bool moe_attr = false;
   int fp8_pair_clusters = 0;
@@ -343,7 +344,7 @@ bsg_status fp8_swap_launch(DeviceState* dev, const void* A, const void* B, const
 }
 
 // tactic 0: one SM per 128 x 256 tile; tactic 1: an SM pair per 256 x 256 tile (cta_group::2);
-// tactics 2, 3: fp8_swap_launch
+// tactics 2, 3: fp8_swap_launch; tactic 4: one SM per 128 x 64 tile (small problems)
 bsg_status fp8_launch(DeviceState* dev, const void* A, const void* B, const float* a_scale, const float* b_scale,
                       const int32_t* m_indices, void* C, int64_t M, int64_t N, int64_t K, int64_t G,
                       bsg_stream_t stream, int tactic) {
@@ -351,6 +352,7 @@ bsg_status fp8_launch(DeviceState* dev, const void* A, const void* B, const floa
     return fp8_swap_launch(dev, A, B, a_scale, b_scale, m_indices, C, M, N, K, G, stream, tactic);
   bsg_status st;
   const int cg = tactic == 1 ? 2 : 1;
+  const bool n64 = tactic == 4;
 
   bsg::Fp8Params p;
   memset(&p, 0, sizeof(p));
@@ -364,9 +366,13 @@ bsg_status fp8_launch(DeviceState* dev, const void* A, const void* B, const floa
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), static_cast<uint64_t>(G)};
     const uint64_t str[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N) * static_cast<uint64_t>(K)};
-    // B rows per CTA and stage: 256 (one SM, 256-column tile) or 128 (each CTA of an SM pair, half of
-    // the pair's 256-column tile)
-    const uint32_t box[3] = {128u, static_cast<uint32_t>(cg == 2 ? bsg::fp8::Cfg<2>::B_BOX_ROWS : bsg::fp8::Cfg<1>::B_BOX_ROWS), 1u};
+    // B rows per CTA and stage: 256 (one SM, 256-column tile), 128 (each CTA of an SM pair, half of
+    // the pair's 256-column tile) or 64 (the 64-column tile)
+    const uint32_t box[3] = {128u,
+                             static_cast<uint32_t>(n64       ? bsg::fp8::Cfg<1, 64>::B_BOX_ROWS
+                                                   : cg == 2 ? bsg::fp8::Cfg<2>::B_BOX_ROWS
+                                                             : bsg::fp8::Cfg<1>::B_BOX_ROWS),
+                             1u};
     const bool oob[3] = {false, true, false};  // an N tail tile is zero-filled, columns masked
     if ((st = encode(&p.tmB, "B", B, 3, dims, str, box, oob, CU_TENSOR_MAP_SWIZZLE_128B)) != BSG_OK) return st;
   }
@@ -378,7 +384,7 @@ bsg_status fp8_launch(DeviceState* dev, const void* A, const void* B, const floa
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.G = static_cast<int>(G);
-  const int bn = cg == 2 ? bsg::fp8::Cfg<2>::BN : bsg::fp8::Cfg<1>::BN;
+  const int bn = n64 ? 64 : (cg == 2 ? bsg::fp8::Cfg<2>::BN : bsg::fp8::Cfg<1>::BN);
   p.n_group = n_group_for(N, K, bn);
   p.timeout_ns = current_timeout();
   p.status = dev->status;
@@ -411,7 +417,16 @@ bsg_status fp8_launch(DeviceState* dev, const void* A, const void* B, const floa
     dev->fp8_attr = true;
   }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  if (cg == 1) {
+  if (n64) {
+    if (!dev->fp8_n64_attr) {
+      e = cudaFuncSetAttribute(bsg::fp8::bsg_fp8_grouped_n64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(bsg::fp8::smem_bytes<1, 64>()));
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(fp8 64-column kernel smem)");
+      dev->fp8_n64_attr = true;
+    }
+    const int grid = bsg_forced_grid(0, grid_for(dev->sm_count, M, N, G, bn));
+    bsg::fp8::bsg_fp8_grouped_n64_kernel<<<grid, bsg::fp8::THREADS, bsg::fp8::smem_bytes<1, 64>(), cs>>>(p);
+  } else if (cg == 1) {
     const int grid = bsg_forced_grid(0, grid_for(dev->sm_count, M, N, G, bn));
     bsg::fp8::bsg_fp8_grouped_kernel<<<grid, bsg::fp8::THREADS, bsg::fp8::smem_bytes<1>(), cs>>>(p);
   } else {

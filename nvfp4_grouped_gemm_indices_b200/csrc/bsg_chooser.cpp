@@ -49,6 +49,7 @@ const Tactic kFp8[] = {
     {"fp8_2sm_m256_n256_s6", 256, 256, 2, 1, 0.45, 0},
     {"fp8_swapab_1sm_n128_t128_s6", 128, 128, 1, 1, 0.24, 1},
     {"fp8_swapab_1sm_n256_t64_s5", 64, 256, 1, 1, 0.23, 1},
+    {"fp8_1sm_m128_n64_s8", 128, 64, 1, 1, 0.19, 0},
 };
 const Tactic kNvfp4[] = {
     {"nvfp4_1sm_m128_n256_s4", 128, 256, 1, 1, 0.52, 0},

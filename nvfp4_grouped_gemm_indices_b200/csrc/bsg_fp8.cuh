@@ -71,17 +71,17 @@ constexpr int NUM_WARPS = WARP_EPI0 + EPI_WARPS;
 constexpr int THREADS = NUM_WARPS * 32;
 constexpr int TMEM_COLS = 512;
 
-template <int CG>
+template <int CG, int BN_ = 256>
 struct Cfg {
-  static constexpr int BN = 256;                         // output columns per unit
-  static constexpr int ACC = TMEM_COLS / BN;              // two TMEM accumulators
+  static constexpr int BN = BN_;                          // output columns per unit: 256, or 64
+  static constexpr int ACC = TMEM_COLS / BN;              // TMEM accumulators: 2 (256) or 8 (64)
   static constexpr int B_BOX_ROWS = BN / CG;              // B rows this CTA loads per stage
   static constexpr int A_BYTES = BM * BK;                 // 16 KB
-  static constexpr int B_BYTES = B_BOX_ROWS * BK;         // 32 KB (CG 1) / 16 KB (CG 2)
-  static constexpr int STAGES = CG == 1 ? 4 : 6;          // 192 KB of ring either way
+  static constexpr int B_BYTES = B_BOX_ROWS * BK;         // 32 KB (CG 1) / 16 KB (CG 2) / 8 KB (64)
+  static constexpr int STAGES = BN == 64 ? 8 : (CG == 1 ? 4 : 6);   // 192 KB of ring in each case
   static constexpr uint32_t STAGE_TX = CG * (A_BYTES + B_BYTES);  // bytes counted on the even CTA
-  static constexpr int EPI_COLS = BN / 4;                 // columns per epilogue warp: 64
-  static constexpr int NB_TILE = BN / 128;                // 128-column scale blocks per tile
+  static constexpr int EPI_COLS = BN / 4;                 // columns per epilogue warp: 64 or 16
+  static constexpr int NB_TILE = BN >= 128 ? BN / 128 : 1;  // 128-column scale blocks per tile
 };
 
 struct ScaleSlot {
@@ -90,33 +90,33 @@ struct ScaleSlot {
   float pad[2];
 };
 
-template <int CG>
+template <int CG, int BN = 256>
 struct alignas(1024) Smem {
-  uint8_t a[Cfg<CG>::STAGES][Cfg<CG>::A_BYTES];
-  uint8_t b[Cfg<CG>::STAGES][Cfg<CG>::B_BYTES];
+  uint8_t a[Cfg<CG, BN>::STAGES][Cfg<CG, BN>::A_BYTES];
+  uint8_t b[Cfg<CG, BN>::STAGES][Cfg<CG, BN>::B_BYTES];
   ScaleSlot sc[SC_STAGES];
-  uint64_t full[Cfg<CG>::STAGES];   // CG 1: own loads; CG 2: (even CTA) both CTAs' loads
-  uint64_t empty[Cfg<CG>::STAGES];  // one MMA commit (multicast to both CTAs of a pair)
+  uint64_t full[Cfg<CG, BN>::STAGES];   // CG 1: own loads; CG 2: (even CTA) both CTAs' loads
+  uint64_t empty[Cfg<CG, BN>::STAGES];  // one MMA commit (multicast to both CTAs of a pair)
   uint64_t sc_full[SC_STAGES];      // 32 cp.async arrivals (one per producer lane)
   uint64_t sc_empty[SC_STAGES];     // EPI_WARPS arrivals
-  uint64_t tmem_full[Cfg<CG>::ACC];   // one MMA commit
-  uint64_t tmem_empty[Cfg<CG>::ACC];  // (even CTA) CG * EPI_WARPS arrivals
+  uint64_t tmem_full[Cfg<CG, BN>::ACC];   // one MMA commit
+  uint64_t tmem_empty[Cfg<CG, BN>::ACC];  // (even CTA) CG * EPI_WARPS arrivals
   uint64_t mma_done;
   UnitQueue<Q> queue;
   uint32_t tmem_base;
   int abort;
 };
 
-template <int CG>
+template <int CG, int BN = 256>
 constexpr size_t smem_bytes() {
-  return sizeof(Smem<CG>) + 1024;  // + alignment slack
+  return sizeof(Smem<CG, BN>) + 1024;  // + alignment slack
 }
 
-template <int CG>
-__device__ __forceinline__ Smem<CG>& smem_ref(uint8_t* raw) {
+template <int CG, int BN = 256>
+__device__ __forceinline__ Smem<CG, BN>& smem_ref(uint8_t* raw) {
   uintptr_t p = reinterpret_cast<uintptr_t>(raw);
   p = (p + 1023) & ~static_cast<uintptr_t>(1023);
-  return *reinterpret_cast<Smem<CG>*>(p);
+  return *reinterpret_cast<Smem<CG, BN>*>(p);
 }
 
 // 4-byte cp.async global -> shared; src_bytes = 0 zero-fills the destination without reading.
@@ -131,12 +131,12 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-template <int CG>
+template <int CG, int BN_ = 256>
 __device__ __forceinline__ void fp8_kernel_body(const Fp8Params& p) {
-  using C = Cfg<CG>;
+  using C = Cfg<CG, BN_>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
-  Smem<CG>& s = smem_ref<CG>(smem_raw);
+  Smem<CG, BN_>& s = smem_ref<CG, BN_>(smem_raw);
   const int warp = warp_idx();
   const int lane = lane_idx();
   const int KB = p.K / BK;
@@ -382,19 +382,29 @@ __device__ __forceinline__ void fp8_kernel_body(const Fp8Params& p) {
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + lane_addr + static_cast<uint32_t>(accp.stage * BN + cg * EPI_COLS);
+        if constexpr (EPI_COLS % 32 == 0) {
 #pragma unroll
-        for (int c = 0; c < EPI_COLS; c += 32) {
-          uint32_t v0[16], v1[16];
-          tmem_ld_x16(taddr + c, v0);
-          tmem_ld_x16(taddr + c + 16, v1);
+          for (int c = 0; c < EPI_COLS; c += 32) {
+            uint32_t v0[16], v1[16];
+            tmem_ld_x16(taddr + c, v0);
+            tmem_ld_x16(taddr + c + 16, v1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              accum[c / 2 + i] = __ffma2_rn(make_float2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1])),
+                                            scale, accum[c / 2 + i]);
+              accum[c / 2 + 8 + i] = __ffma2_rn(
+                  make_float2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1])), scale, accum[c / 2 + 8 + i]);
+            }
+          }
+        } else {                                         // 16 columns per warp (the 64-column tile)
+          uint32_t v0[16];
+          tmem_ld_x16(taddr, v0);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            accum[c / 2 + i] = __ffma2_rn(make_float2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1])),
-                                          scale, accum[c / 2 + i]);
-            accum[c / 2 + 8 + i] = __ffma2_rn(
-                make_float2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1])), scale, accum[c / 2 + 8 + i]);
-          }
+          for (int i = 0; i < 8; ++i)
+            accum[i] = __ffma2_rn(make_float2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1])), scale,
+                                  accum[i]);
         }
         tc_fence_before();
         __syncwarp();
@@ -450,6 +460,13 @@ __global__ void __launch_bounds__(THREADS, 1) bsg_fp8_grouped_kernel(const __gri
 // Launched as clusters of 2 CTAs (grid a multiple of 2).
 __global__ void __launch_bounds__(THREADS, 1) bsg_fp8_grouped_2sm_kernel(const __grid_constant__ Fp8Params p) {
   fp8_kernel_body<2>(p);
+}
+
+// The 64-column tile for small problems: four times as many units as the 256-column tile, each a
+// quarter of the MMA, promotion and store work per K block, eight accumulators and an eight-stage
+// ring; on a grid that does not fill the GPU its units finish sooner.
+__global__ void __launch_bounds__(THREADS, 1) bsg_fp8_grouped_n64_kernel(const __grid_constant__ Fp8Params p) {
+  fp8_kernel_body<1, 64>(p);
 }
 
 }  // namespace fp8

@@ -15,8 +15,9 @@ from gpu_util import (SENTINEL, DevWorkload, bits, compare, oracle_rows, routed_
 
 pytestmark = pytest.mark.gpu
 
-FP8_TACTICS = [0, 1, 2, 3]  # 0: one SM per 128 x 256 tile; 1: an SM pair per 256 x 256 tile (cta_group::2);
-# 2, 3: operand-swapped tiles (128 or 256 output columns x a chunk of at most 128 or 64 tokens)
+FP8_TACTICS = [0, 1, 2, 3, 4]  # 0: one SM per 128 x 256 tile; 1: an SM pair per 256 x 256 tile (cta_group::2);
+# 2, 3: operand-swapped tiles (128 or 256 output columns x a chunk of at most 128 or 64 tokens);
+# 4: one SM per 128 x 64 tile (small problems)
 
 
 @pytest.fixture(params=FP8_TACTICS, ids=lambda t: f"tactic{t}")
