@@ -204,7 +204,8 @@ uint64_t bsg_set_wait_timeout_ns(uint64_t ns);
  * tile; 2, 3 = operand-swapped tiles for experts with few rows (128 or 256 output columns x a chunk
  * of at most 128 or 64 of one expert's rows; the page "[onnxruntime] ONNX Runtime: Blackwell
  * (SM120+)에서 NVFP4 QMoE를 위한 네이티브 FP4xFP4 Prefill 최적화", section 1, keeps decode shapes on a
- * path of their own).  NVFP4 tactics: 0 = one SM, 1 = an SM pair.  Every tactic computes the same
+ * path of their own); 4 = one SM per 128-row window segment x 64 columns (small problems, the
+ * small-launch shapes of the FP8 page's section 2 table).  NVFP4 tactics: 0 = one SM, 1 = an SM pair.  Every tactic computes the same
  * result within the stated tolerance.
  */
 int bsg_num_tactics(int kind);
