@@ -165,9 +165,16 @@ def test_chooser_score_follows_the_page_formula(lib):
         # measured: the row tile streams the decode shape fastest, and the prefill shape too
         assert bsg.bsg_choose_tactic(0, 512, 4096, 7168, 64, 148) == 0
         assert bsg.bsg_choose_tactic(0, 8192, 4096, 7168, 8, 148) not in swaps
-        # the small 4-expert shape (runs of ~128 rows, 256 columns) fills two swapped units per segment
-        # where the row tile has one: the swapped 128-column tile ranks first (measured: a tie)
-        assert bsg.bsg_choose_tactic(0, 512, 256, 512, 4, 148) == swaps[0]
+    n64 = [t for t, nm in enumerate(names) if "_n64_" in nm]
+    if n64:
+        # small problems: the 64-column tile gives a 4-expert, 512-row, 256-column launch four units per
+        # segment where the 256-column tile has one; it ranks first there and on the FP8 page's two
+        # shapes (measured fastest on all three), and last on the prefill shape
+        assert bsg.bsg_choose_tactic(0, 512, 256, 512, 4, 148) == n64[0]
+        assert bsg.bsg_choose_tactic(0, 65, 128, 128, 2, 148) == n64[0]
+        assert bsg.bsg_choose_tactic(0, 777, 256, 512, 8, 148) == n64[0]
+        assert bsg.bsg_choose_tactic(0, 8192, 4096, 7168, 8, 148) != n64[0]
+        assert bsg.bsg_choose_tactic(0, 512, 4096, 7168, 64, 148) != n64[0]
     assert bsg.bsg_tactic_score(0, 99, 1, 64, 128, 1, 148) == 0.0
 
 
