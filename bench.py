@@ -223,10 +223,25 @@ def visible_gpu_index(local_rank):
 # ----------------------------------------------------------------------------- kernel source hash
 
 
-def kernel_source_hash():
+# The device code each workload's counters depend on: its kernels' own headers, the shared PTX
+# wrappers and scheduler, and the tactic chooser that picks among them.  A change anywhere else (host
+# entry points, another kernel family) leaves the recorded counters valid.
+KERNEL_SOURCES = {
+    "fp8": ["bsg_fp8.cuh", "bsg_fp8_swap.cuh", "bsg_sched.cuh", "bsg_ptx.cuh", "bsg_chooser.cpp"],
+    "nvfp4": ["bsg_nvfp4.cuh", "bsg_sched.cuh", "bsg_ptx.cuh", "bsg_chooser.cpp"],
+    "quant": ["bsg_quant.cuh"],
+    "moe": ["bsg_moe.cuh"],
+}
+
+
+def kernel_family(workload_name):
+    return workload_name.split("_", 1)[0]
+
+
+def kernel_source_hash(family):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "nvfp4_grouped_gemm_indices_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(KERNEL_SOURCES[family]):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode())
             h.update(fh.read())
@@ -235,14 +250,14 @@ def kernel_source_hash():
 
 def recorded_profile(workload_name):
     """The committed ncu figures of one workload's kernel (profiles/traffic.json): DRAM bytes per
-    launch and tensor-pipe activity, if taken on the current kernel sources; else {}."""
+    launch and tensor-pipe activity, if taken on the current sources of that kernel; else {}."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return {}
     with open(p) as f:
         d = json.load(f)
     e = d.get(workload_name)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel_family(workload_name)):
         return {}
     return e
 
