@@ -57,6 +57,8 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--sweep", action="store_true",
                     help="time every tactic on a set of shapes and compare with the chooser's pick")
+    ap.add_argument("--moe-only", action="store_true",
+                    help="time only the MoE expand permutation (three routing sizes)")
     ap.add_argument("--quant-only", action="store_true",
                     help="time only the activation quantisers (one JSON line each) -- for profiling")
     return ap.parse_args(argv)
@@ -472,9 +474,11 @@ def time_quantiser(kind, M, K, peaks, steps=50, warmup=5):
 
 
 def time_moe_permute(T, top_k, G, peaks, steps=50, warmup=5):
-    """The MoE expand permutation (three kernel launches: per-tile counts, scan, stable scatter) on a
-    Zipf-skewed routing of T tokens x top_k choices over G experts.  Integer work bound by the
-    latency of its dependent steps; reported with the HBM bytes it must move."""
+    """The MoE expand permutation (one single-CTA launch up to 2^16 entries over at most 1024 experts,
+    else three: per-tile counts, scan, stable scatter) on a Zipf-skewed routing of T tokens x top_k
+    choices over G experts.  Integer work bound by the latency of its dependent steps; reported with
+    the HBM bytes it must move, as GPU time per call (CUDA-graph replay of `steps` calls) and as the
+    rate of calls issued one by one from Python."""
     import torch
     import nvfp4_grouped_gemm_indices_b200 as bsg
     g = torch.Generator(device="cuda").manual_seed(T * 131 + G)
@@ -482,27 +486,44 @@ def time_moe_permute(T, top_k, G, peaks, steps=50, warmup=5):
     ids = torch.multinomial((ranks / ranks.sum()).float(), T * top_k, replacement=True, generator=g)
     ids = ids.to(torch.int32).view(T, top_k)
     n = T * top_k
-    ws = torch.empty(max(16, bsg.bsg_moe_permute_workspace_size(T, top_k, G)), dtype=torch.uint8, device="cuda")
+    need = bsg.bsg_moe_permute_workspace_size(T, top_k, G)
+    ws = torch.empty(max(16, need), dtype=torch.uint8, device="cuda")
     outs = [torch.empty(n, dtype=torch.int32, device="cuda"), torch.empty(n, dtype=torch.int32, device="cuda"),
             torch.empty((T, top_k), dtype=torch.int32, device="cuda"),
             torch.empty(G + 1, dtype=torch.int32, device="cuda")]
-    stream = torch.cuda.current_stream()
-    launch = lambda: bsg.bsg_moe_permute(ids, T, top_k, G, *outs, ws, ws.numel(), stream.cuda_stream)
-    for _ in range(warmup):
-        launch()
-    torch.cuda.synchronize()
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        launch()
-    b.record(stream)
-    b.synchronize()
-    per = a.elapsed_time(b) / 1e3 / steps
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        launch = lambda: bsg.bsg_moe_permute(ids, T, top_k, G, *outs, ws, ws.numel(), side.cuda_stream)
+        for _ in range(warmup):
+            launch()
+        side.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(side)
+        for _ in range(steps):
+            launch()
+        b.record(side)
+        b.synchronize()
+        per_host = a.elapsed_time(b) / 1e3 / steps
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            for _ in range(steps):
+                launch()
+        graph.replay()
+        side.synchronize()
+        a.record(side)
+        graph.replay()
+        b.record(side)
+        b.synchronize()
+        per = a.elapsed_time(b) / 1e3 / steps
+        del graph
     nbytes = 2 * 4 * n + 3 * 4 * n + 4 * (G + 1)      # ids read twice; src, m_indices, dst written
-    return {"us_per_launch": round(per * 1e6, 2), "kernel_launches": 3,
+    return {"us_per_launch": round(per * 1e6, 2), "us_per_call_issued_from_python": round(per_host * 1e6, 2),
+            "kernel_launches": 1 if need == 0 else 3,
             "hbm_bytes": nbytes, "achieved_gbs": round(nbytes / per / 1e9, 1),
-            "note": "latency-bound integer work; back-to-back launches, inputs L2-resident"}
+            "note": "latency-bound integer work; GPU time per call from a CUDA graph of "
+                    f"{steps} calls, inputs L2-resident"}
 
 
 def cpu_baseline(w, seconds):
@@ -633,6 +654,7 @@ def run_bsg(args):
         also["quant_nvfp4_rows_gather_m65536_k8192"] = time_quantiser("nvfp4", 65536, 8192, peaks)
         also["moe_permute_t8192_k8_g64"] = time_moe_permute(8192, 8, 64, peaks)
         also["moe_permute_t64_k8_g64"] = time_moe_permute(64, 8, 64, peaks)
+        also["moe_permute_t65536_k8_g256"] = time_moe_permute(65536, 8, 256, peaks)
         line["also"] = also
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -689,6 +711,15 @@ def run_quant_only(args):
     for kind, M, K in (("fp8", 8192, 7168), ("nvfp4", 65536, 8192)):
         d = time_quantiser(kind, M, K, peaks, steps=max(1, args.steps), warmup=max(1, args.warmup))
         print(json.dumps({"kernel": f"quant_{kind}_rows_gather_m{M}_k{K}", **d}), flush=True)
+
+
+def run_moe_only(args):
+    import torch
+    torch.cuda.set_device(0)
+    peaks, _ = load_peaks()
+    for T, top_k, G in ((8192, 8, 64), (64, 8, 64), (65536, 8, 256)):
+        d = time_moe_permute(T, top_k, G, peaks, steps=max(1, args.steps), warmup=max(1, args.warmup))
+        print(json.dumps({"kernel": f"moe_permute_t{T}_k{top_k}_g{G}", **d}), flush=True)
 
 
 def sweep_shapes():
@@ -754,6 +785,9 @@ def main(argv=None):
         return
     if args.quant_only:
         run_quant_only(args)
+        return
+    if args.moe_only:
+        run_moe_only(args)
         return
     if args.impl == "reference":
         run_reference(args)

@@ -139,11 +139,14 @@ bsg_status bsg_quantize_nvfp4_rows(const void* X, const int32_t* src_rows, const
  * expert_offsets  int32 [G + 1]     output: start of each expert's run; [G] = rows placed.
  * workspace       device scratch of at least bsg_moe_permute_workspace_size() bytes, 16-byte
  *                 aligned, owned by the caller; its contents need not be initialised and are
- *                 overwritten.  Calls that share a workspace must not overlap on the GPU.
+ *                 overwritten.  Calls that share a workspace must not overlap on the GPU.  When
+ *                 that size is 0 the workspace is not used and may be null.
  * Contract: T >= 1, 1 <= top_k <= 256, T * top_k <= 2^24, 1 <= G <= 4096; the int32 arrays 4-byte
- *           aligned.  Asynchronous on `stream`; nothing is allocated.  Three kernel launches.
- * bsg_moe_permute_workspace_size() writes the scratch size for (T, top_k, G) to *bytes (at most
- * 16 MiB) or returns an error for sizes outside the contract; it touches no GPU.
+ *           aligned.  Asynchronous on `stream`; nothing is allocated.  One kernel launch (one CTA,
+ *           no scratch) when T * top_k <= 4096 and G <= 1024, three launches otherwise.
+ * bsg_moe_permute_workspace_size() writes the scratch size for (T, top_k, G) to *bytes (0 for the
+ * one-launch sizes, else 4 * G * min(512, ceil(T * top_k / 256)) up to rounding of the tiles, at most
+ * 8 MiB) or returns an error for sizes outside the contract; it touches no GPU.
  */
 bsg_status bsg_moe_permute_workspace_size(int64_t T, int64_t top_k, int64_t G, size_t* bytes);
 bsg_status bsg_moe_permute(const int32_t* expert_ids, int64_t T, int64_t top_k, int64_t G, int32_t* src_rows,
@@ -160,9 +163,10 @@ bsg_status bsg_moe_permute(const int32_t* expert_ids, int64_t T, int64_t top_k, 
  *
  * The scratch is a fixed 2 MiB array that the library's device image carries on every GPU that loads
  * it, for as long as the process lives.  Limit: the sizes (T, top_k, G) whose
- * bsg_moe_permute_workspace_size() is at most 2 MiB -- for example T * top_k up to 2^21 entries with
- * G = 64, 2^19 with G = 256, 2^14 with G = 4096; larger sizes return BSG_ERR_UNSUPPORTED_SHAPE with a
- * message and launch nothing.  The first call on a device also looks up that device's copy of the
+ * bsg_moe_permute_workspace_size() is at most 2 MiB -- every size with G <= 1024, and with more experts
+ * T * top_k up to 65536 entries for G = 2048 or 32768 for G = 4096; larger sizes return
+ * BSG_ERR_UNSUPPORTED_SHAPE with a message and launch nothing.  The first call on a device also looks
+ * up that device's copy of the
  * array (with the device current), so make that first call before capturing any stream.
  * Every call on a device shares the one array and leaves its last contents behind; the kernels
  * overwrite every counter before they read it, so nothing needs clearing between calls, but calls

@@ -362,7 +362,8 @@ def nvfp4_gemm(A, B, sfa, sfb, alpha, m_indices, out=None, stream=None):
 def moe_permute(expert_ids, G, stream=None):
     """expert_ids int32 [T, top_k] (CUDA) -> (src_rows int32 [T*top_k], m_indices int32 [T*top_k],
     dst_rows int32 [T, top_k], expert_offsets int32 [G+1]): the expert-grouped layout of the routing
-    entries (see bsg_moe_permute); the scratch is a torch allocation made here."""
+    entries (see bsg_moe_permute); the scratch, when the sizes need one, is a torch allocation made
+    here."""
     import torch
     _need(expert_ids, torch.int32, "expert_ids", 2)
     T, top_k = expert_ids.shape
@@ -370,12 +371,12 @@ def moe_permute(expert_ids, G, stream=None):
     dev = _same_device((("expert_ids", expert_ids),), stream)
     with torch.cuda.device(dev):
         nbytes = bsg_moe_permute_workspace_size(T, top_k, G)
-        ws = torch.empty(max(16, nbytes), dtype=torch.uint8, device=dev)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
         src = torch.empty(n, dtype=torch.int32, device=dev)
         mi = torch.empty(n, dtype=torch.int32, device=dev)
         dst = torch.empty((T, top_k), dtype=torch.int32, device=dev)
         off = torch.empty(G + 1, dtype=torch.int32, device=dev)
-        bsg_moe_permute(expert_ids, T, top_k, G, src, mi, dst, off, ws, ws.numel(), stream)
+        bsg_moe_permute(expert_ids, T, top_k, G, src, mi, dst, off, ws, nbytes, stream)
     return src, mi, dst, off
 
 

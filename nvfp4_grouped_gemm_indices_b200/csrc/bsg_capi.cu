@@ -768,6 +768,7 @@ namespace {
 // Tiling of the MoE permutation: tiles of at least MIN_TILE entries (multiples of 32), at most
 // cap_ints / G of them, so that the scratch (tiles x G int32 counters) stays within cap_ints.
 struct MoePlan {
+  bool fused = false;   // the single-CTA kernel (no scratch)
   int tile = 0;
   int tiles = 0;
   size_t scratch_bytes = 0;
@@ -777,8 +778,16 @@ constexpr int64_t kMoeWorkspaceCapInts = 1ll << 22;  // 16 MiB of counters at mo
 
 MoePlan moe_plan(int64_t n, int64_t G, int64_t cap_ints) {
   MoePlan pl;
+  if (n <= bsg::moe::FUSED_MAX_N && G <= bsg::moe::FUSED_MAX_G) {
+    const int64_t per = (n + bsg::moe::FUSED_WARPS - 1) / bsg::moe::FUSED_WARPS;
+    pl.fused = true;
+    pl.tile = static_cast<int>((per + 31) / 32 * 32);
+    pl.tiles = bsg::moe::FUSED_WARPS;
+    return pl;
+  }
   int64_t tiles = (n + bsg::moe::MIN_TILE - 1) / bsg::moe::MIN_TILE;
   if (tiles < 1) tiles = 1;
+  if (tiles > bsg::moe::MAX_TILES) tiles = bsg::moe::MAX_TILES;
   if (tiles * G > cap_ints) tiles = cap_ints / G > 1 ? cap_ints / G : 1;
   int64_t tile = (n + tiles - 1) / tiles;
   tile = (tile + 31) / 32 * 32;
@@ -812,7 +821,8 @@ bsg_status moe_check(const int32_t* expert_ids, int64_t T, int64_t top_k, int64_
   return BSG_OK;
 }
 
-// The three kernels of the permutation on `stream`, with `scratch` (pl.scratch_bytes, 4-byte aligned).
+// The permutation on `stream`: the single-CTA kernel, or the three kernels with `scratch`
+// (pl.scratch_bytes, 4-byte aligned).
 bsg_status moe_launch(DeviceState* dev, const int32_t* expert_ids, int64_t T, int64_t top_k, int64_t G,
                       int32_t* src_rows, int32_t* m_indices, int32_t* dst_rows, int32_t* expert_offsets,
                       int32_t* scratch, const MoePlan& pl, bsg_stream_t stream) {
@@ -823,6 +833,9 @@ bsg_status moe_launch(DeviceState* dev, const int32_t* expert_ids, int64_t T, in
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(moe count kernel smem)");
     e = cudaFuncSetAttribute(bsg::moe::bsg_moe_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(moe scatter kernel smem)");
+    const int fused_smem = bsg::moe::FUSED_WARPS * bsg::moe::FUSED_MAX_G * static_cast<int>(sizeof(int32_t));
+    e = cudaFuncSetAttribute(bsg::moe::bsg_moe_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fused_smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(moe single-CTA kernel smem)");
     dev->moe_attr = true;
   }
   bsg::moe::Params p;
@@ -839,10 +852,19 @@ bsg_status moe_launch(DeviceState* dev, const int32_t* expert_ids, int64_t T, in
   p.tile = pl.tile;
   p.tiles = pl.tiles;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (pl.fused) {
+    const size_t smem = static_cast<size_t>(bsg::moe::FUSED_WARPS) * static_cast<size_t>(G) * sizeof(int32_t);
+    bsg::moe::bsg_moe_fused_kernel<<<1, bsg::moe::FUSED_THREADS, smem, cs>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the MoE permutation kernel");
+    return BSG_OK;
+  }
   const int blocks = (pl.tiles + bsg::moe::WARPS - 1) / bsg::moe::WARPS;
   const size_t tile_smem = static_cast<size_t>(bsg::moe::WARPS) * static_cast<size_t>(G) * sizeof(int32_t);
   bsg::moe::bsg_moe_count_kernel<<<blocks, bsg::moe::THREADS, tile_smem, cs>>>(p);
-  bsg::moe::bsg_moe_scan_kernel<<<1, bsg::moe::SCAN_THREADS, static_cast<size_t>(G) * sizeof(int32_t), cs>>>(p);
+  const int64_t scan_segments = G <= bsg::moe::SCAN_THREADS ? bsg::moe::SCAN_THREADS / G : 1;
+  const size_t scan_smem = static_cast<size_t>(scan_segments * G + G) * sizeof(int32_t);   // <= 32 KiB
+  bsg::moe::bsg_moe_scan_kernel<<<1, bsg::moe::SCAN_THREADS, scan_smem, cs>>>(p);
   bsg::moe::bsg_moe_scatter_kernel<<<blocks, bsg::moe::THREADS, tile_smem, cs>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launch of the MoE permutation kernels");
@@ -869,10 +891,10 @@ bsg_status bsg_moe_permute(const int32_t* expert_ids, int64_t T, int64_t top_k, 
   bsg_status st = moe_check(expert_ids, T, top_k, G, src_rows, m_indices, dst_rows, expert_offsets);
   if (st != BSG_OK) return st;
   const MoePlan pl = moe_plan(T * top_k, G, kMoeWorkspaceCapInts);
-  if (!workspace || workspace_bytes < pl.scratch_bytes)
+  if (pl.scratch_bytes > 0 && (!workspace || workspace_bytes < pl.scratch_bytes))
     return fail(BSG_ERR_INVALID_ARG, "workspace of %zu bytes is missing or smaller than the %zu bytes needed",
                 workspace_bytes, pl.scratch_bytes);
-  if (!aligned(workspace, 16)) return fail(BSG_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  if (workspace && !aligned(workspace, 16)) return fail(BSG_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
   DeviceState* dev = nullptr;
   if ((st = device_state(&dev)) != BSG_OK) return st;
   return moe_launch(dev, expert_ids, T, top_k, G, src_rows, m_indices, dst_rows, expert_offsets,

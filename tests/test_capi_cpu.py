@@ -291,12 +291,21 @@ def test_fp8_wrapper_rejects_a_wrong_shaped_out_before_any_launch(monkeypatch):
 
 
 def test_moe_permute_workspace_size(lib):
-    # tiles of at least 256 entries (multiples of 32), one row of G int32 counters per tile
+    # up to 4096 entries over at most 1024 experts: one CTA, counters in shared memory, no scratch
+    assert bsg.bsg_moe_permute_workspace_size(1, 1, 1) == 0
+    assert bsg.bsg_moe_permute_workspace_size(100, 3, 64) == 0
+    assert bsg.bsg_moe_permute_workspace_size(512, 8, 1024) == 0
+    # otherwise tiles of at least 256 entries (multiples of 32), at most 512 tiles, one row of G int32
+    # counters per tile: 65536 entries -> 256 tiles; 65544 -> 257 tiles of 256; 300 entries over 2048
+    # experts -> 2 tiles of 160; 4097 entries -> 17 tiles
     assert bsg.bsg_moe_permute_workspace_size(8192, 8, 8) == 256 * 8 * 4
-    assert bsg.bsg_moe_permute_workspace_size(1, 1, 1) == 4
-    assert bsg.bsg_moe_permute_workspace_size(100, 3, 64) == 2 * 64 * 4
-    # capped at 2^22 counters (16 MiB): G = 4096 allows 1024 tiles
-    assert bsg.bsg_moe_permute_workspace_size(1 << 21, 8, 4096) == 1024 * 4096 * 4
+    assert bsg.bsg_moe_permute_workspace_size(8193, 8, 8) == 257 * 8 * 4
+    assert bsg.bsg_moe_permute_workspace_size(100, 3, 2048) == 2 * 2048 * 4
+    assert bsg.bsg_moe_permute_workspace_size(4097, 1, 8) == 17 * 8 * 4
+    assert bsg.bsg_moe_permute_workspace_size(65536, 1, 1024) == 256 * 1024 * 4
+    # 2^24 entries: 512 tiles of 32768 whatever G is
+    assert bsg.bsg_moe_permute_workspace_size(1 << 21, 8, 64) == 512 * 64 * 4
+    assert bsg.bsg_moe_permute_workspace_size(1 << 21, 8, 4096) == 512 * 4096 * 4
     for T, k, G, needle in ((0, 1, 4, "T = 0"), (4, 0, 4, "top_k = 0"), (4, 300, 4, "256"),
                             (1 << 22, 8, 4, "2^24"), (4, 2, 0, "G = 0"), (4, 2, 5000, "4096")):
         with pytest.raises(bsg.BsgError) as ei:
@@ -315,7 +324,8 @@ def test_moe_permute_workspace_size(lib):
     (dict(G=0), bsg.BSG_ERR_UNSUPPORTED_SHAPE, "G = 0"),
 ])
 def test_moe_permute_argument_errors(lib, kw, status, needle):
-    a = dict(expert_ids=FAKE, T=512, top_k=2, G=8, src_rows=FAKE, m_indices=FAKE, dst_rows=FAKE,
+    # 1024 entries over 2048 experts: the three-launch path, 32 KB of scratch
+    a = dict(expert_ids=FAKE, T=512, top_k=2, G=2048, src_rows=FAKE, m_indices=FAKE, dst_rows=FAKE,
              expert_offsets=FAKE, workspace=FAKE, workspace_bytes=1 << 20)
     a.update(kw)
     with pytest.raises(bsg.BsgError) as ei:

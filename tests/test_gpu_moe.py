@@ -55,6 +55,9 @@ def check(ids, G, got):
 @pytest.mark.parametrize("T,top_k,G,invalid,zipf", [
     (1, 1, 1, 0.0, False), (37, 3, 5, 0.2, False), (8192, 8, 8, 0.0, False), (4096, 6, 256, 0.0, True),
     (1000, 2, 4096, 0.05, False), (50, 4, 3, 1.0, False), (65536, 8, 64, 0.01, True), (257, 1, 2, 0.0, False),
+    # the single-CTA path's limits (4096 entries, 1024 experts) and the first sizes past them
+    (512, 8, 1024, 0.01, True), (9, 7, 1024, 0.0, False), (4097, 1, 8, 0.0, True), (64, 2, 1025, 0.1, False),
+    (2048, 32, 1024, 0.01, True), (1 << 18, 1, 5, 0.0, True),
 ])
 def test_permute_bit_exact(T, top_k, G, invalid, zipf):
     ids = make_ids(T, top_k, G, seed=T * 7 + G, invalid=invalid, zipf=zipf)
@@ -62,28 +65,30 @@ def test_permute_bit_exact(T, top_k, G, invalid, zipf):
 
 
 def test_permute_largest_size():
-    """T * top_k = 2^24 entries over 4096 experts: the largest tiles the 16 MiB scratch allows."""
+    """T * top_k = 2^24 entries over 4096 experts: 512 tiles of 32768 entries (8 MiB of counters)."""
     T, top_k, G = 1 << 21, 8, 4096
     ids = make_ids(T, top_k, G, seed=5, invalid=0.001, zipf=True)
     check(ids, G, run_permute(ids, G))
 
 
 def test_permute_calls_in_a_row_share_the_workspace():
-    G = 32
-    ws = torch.empty(bsg.bsg_moe_permute_workspace_size(3000, 4, G), dtype=torch.uint8, device="cuda")
+    G = 32                                   # 80000 entries: the three-launch path, with scratch
+    ws = torch.empty(bsg.bsg_moe_permute_workspace_size(20000, 4, G), dtype=torch.uint8, device="cuda")
+    assert ws.numel() > 0
     for seed in range(3):
-        ids = make_ids(3000, 4, G, seed=seed, invalid=0.1)
+        ids = make_ids(20000, 4, G, seed=seed, invalid=0.1)
         check(ids, G, run_permute(ids, G, ws=ws, garbage=False))
 
 
-def test_permute_graph_replay_sees_new_routing():
+@pytest.mark.parametrize("T", [500, 20000])
+def test_permute_graph_replay_sees_new_routing(T):
     """No allocation and no host read in the call: it captures into a CUDA graph, and a replay after
-    the routing changed in place gives the new permutation."""
-    T, top_k, G = 2048, 4, 16
+    the routing changed in place gives the new permutation (single-CTA and three-launch sizes)."""
+    top_k, G = 4, 16
     n = T * top_k
     ids0 = make_ids(T, top_k, G, seed=1)
     e = torch.from_numpy(ids0).cuda()
-    ws = torch.empty(bsg.bsg_moe_permute_workspace_size(T, top_k, G), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(max(16, bsg.bsg_moe_permute_workspace_size(T, top_k, G)), dtype=torch.uint8, device="cuda")
     outs = [torch.empty(n, dtype=torch.int32, device="cuda"), torch.empty(n, dtype=torch.int32, device="cuda"),
             torch.empty((T, top_k), dtype=torch.int32, device="cuda"),
             torch.empty(G + 1, dtype=torch.int32, device="cuda")]
