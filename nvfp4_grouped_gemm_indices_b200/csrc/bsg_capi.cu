@@ -862,12 +862,30 @@ bsg_status moe_launch(DeviceState* dev, const int32_t* expert_ids, int64_t T, in
   const int blocks = (pl.tiles + bsg::moe::WARPS - 1) / bsg::moe::WARPS;
   const size_t tile_smem = static_cast<size_t>(bsg::moe::WARPS) * static_cast<size_t>(G) * sizeof(int32_t);
   bsg::moe::bsg_moe_count_kernel<<<blocks, bsg::moe::THREADS, tile_smem, cs>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the MoE count kernel");
   const int64_t scan_segments = G <= bsg::moe::SCAN_THREADS ? bsg::moe::SCAN_THREADS / G : 1;
   const size_t scan_smem = static_cast<size_t>(scan_segments * G + G) * sizeof(int32_t);   // <= 32 KiB
-  bsg::moe::bsg_moe_scan_kernel<<<1, bsg::moe::SCAN_THREADS, scan_smem, cs>>>(p);
-  bsg::moe::bsg_moe_scatter_kernel<<<blocks, bsg::moe::THREADS, tile_smem, cs>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "launch of the MoE permutation kernels");
+  // the scan and scatter kernels start their launch while the previous kernel runs and wait for it
+  // on the device (programmatic dependent launch)
+  cudaLaunchAttribute la[1];
+  la[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  la[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t lc;
+  memset(&lc, 0, sizeof(lc));
+  lc.stream = cs;
+  lc.attrs = la;
+  lc.numAttrs = 1;
+  lc.gridDim = dim3(1, 1, 1);
+  lc.blockDim = dim3(bsg::moe::SCAN_THREADS, 1, 1);
+  lc.dynamicSmemBytes = scan_smem;
+  e = cudaLaunchKernelEx(&lc, bsg::moe::bsg_moe_scan_kernel, p);
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the MoE scan kernel");
+  lc.gridDim = dim3(blocks, 1, 1);
+  lc.blockDim = dim3(bsg::moe::THREADS, 1, 1);
+  lc.dynamicSmemBytes = tile_smem;
+  e = cudaLaunchKernelEx(&lc, bsg::moe::bsg_moe_scatter_kernel, p);
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the MoE scatter kernel");
   return BSG_OK;
 }
 

@@ -61,6 +61,13 @@ struct Params {
   int tile, tiles;
 };
 
+// Programmatic dependent launch: the scan and scatter kernels are launched while their predecessor
+// still runs, so their launch latency overlaps it; `dependency_wait` blocks until the predecessor
+// grid has completed and its memory writes are visible, `allow_dependents` lets the next grid start
+// its launch early.
+__device__ __forceinline__ void dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ int32_t expert_at(const Params& p, long long i) {
   const int32_t g = __ldg(p.expert_ids + i);
   return (g >= 0 && g < p.G) ? g : -1;
@@ -73,6 +80,7 @@ __global__ void __launch_bounds__(THREADS) bsg_moe_count_kernel(const __grid_con
   const int wib = threadIdx.x >> 5;
   const int w = blockIdx.x * WARPS + wib;
   int32_t* row = moe_smem + static_cast<size_t>(wib) * p.G;
+  allow_dependents();
   if (w >= p.tiles) return;                              // warp-uniform
   for (int g = lane; g < p.G; g += 32) row[g] = 0;
   __syncwarp();
@@ -108,6 +116,8 @@ __global__ void __launch_bounds__(SCAN_THREADS) bsg_moe_scan_kernel(const __grid
   const int G = p.G;
   const int S = G <= SCAN_THREADS ? SCAN_THREADS / G : 1;
   const int seg = (p.tiles + S - 1) / S;
+  allow_dependents();
+  dependency_wait();                                     // the count kernel's rows are complete
   int32_t* seg_sum = moe_smem;                          // [S][G]
   int32_t* start = moe_smem + S * G;                     // [G]
   // 1. each (segment, expert) column's sum
@@ -190,6 +200,7 @@ __global__ void __launch_bounds__(THREADS) bsg_moe_scatter_kernel(const __grid_c
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
   const int w = blockIdx.x * WARPS + wib;
+  dependency_wait();                                     // the scan kernel's positions are complete
   // the unused tail [placed, n): -1 in both expanded maps (grid-stride over the whole grid)
   {
     const long long placed = __ldg(p.expert_offsets + p.G);
