@@ -510,6 +510,13 @@ bsg_status nvfp4_launch(DeviceState* dev, const void* A, const void* B, const vo
     const bool oob[3] = {false, true, false};
     if ((st = encode(&p.tmSFB, "sfb", sfb, 3, dims, str, box, oob, CU_TENSOR_MAP_SWIZZLE_NONE)) != BSG_OK) return st;
   }
+  {
+    const uint64_t dims[2] = {2 * static_cast<uint64_t>(N), static_cast<uint64_t>(M)};
+    const uint64_t str[1] = {2 * static_cast<uint64_t>(N)};
+    const uint32_t box[2] = {128u, 32u};
+    const bool oob[2] = {true, true};
+    if ((st = encode(&p.tmC, "C", C, 2, dims, str, box, oob, CU_TENSOR_MAP_SWIZZLE_128B)) != BSG_OK) return st;
+  }
   p.alpha = alpha;
   p.m_indices = m_indices;
   p.C = static_cast<__nv_bfloat16*>(C);

@@ -49,6 +49,7 @@ struct Nvfp4Params {
   CUtensorMap tmB;  // uint8 [G, N, K/2]: dims {K/2, N, G}, box {128, BN, 1}, 128B swizzle
   CUtensorMap tmSFA;  // uint8 [M, K/16]:    dims {K/16, M},    box {16, 128}
   CUtensorMap tmSFB;  // uint8 [G, N, K/16]: dims {K/16, N, G}, box {16, BN, 1}
+  CUtensorMap tmC;    // bf16 C as bytes [M, 2N]: dims {2N, M}, box {128, 32}, 128B swizzle
   const float* alpha;
   const int* m_indices;
   __nv_bfloat16* C;
@@ -60,6 +61,24 @@ struct Nvfp4Params {
 };
 
 namespace nvfp4 {
+
+// TMA store of a tile from shared memory (bulk-group completion) and its helpers (the C epilogue of
+// the pair kernel).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
 
 constexpr int BM = 128;                  // rows per CTA
 constexpr int BN = 256;                  // output columns per unit (both variants)
@@ -93,6 +112,8 @@ struct alignas(1024) Smem {
   uint8_t a[Cfg<CG>::STAGES][A_BYTES];
   uint8_t b[Cfg<CG>::STAGES][Cfg<CG>::B_BYTES];
   alignas(128) uint8_t sf[Cfg<CG>::STAGES][SFA_BYTES + SFB_BYTES];  // raw row-major scale bytes (TMA)
+  // (pair kernel) each epilogue warp's C staging tile: 32 rows x 64 BF16, 128B-swizzled for the TMA store
+  alignas(1024) uint8_t stage_c[CG == 2 ? EPI_WARPS : 1][CG == 2 ? 32 * 128 : 16];
   uint64_t full[Cfg<CG>::STAGES];    // (even CTA) A/B bytes + FULL_ARRIVALS arrivals
   uint64_t sf_raw[Cfg<CG>::STAGES];  // this CTA's raw scale bytes landed (1 arrival + bytes)
   uint64_t empty[Cfg<CG>::STAGES];   // 1 MMA commit: the stage's smem and TMEM scale slot are free
@@ -108,6 +129,7 @@ template <int CG>
 constexpr size_t smem_bytes() {
   return sizeof(Smem<CG>) + 1024;  // + alignment slack
 }
+static_assert(smem_bytes<2>() <= 232448, "pair kernel shared memory above 227 KB");
 
 template <int CG>
 __device__ __forceinline__ Smem<CG>& smem_ref(uint8_t* raw) {
@@ -381,7 +403,27 @@ __device__ __forceinline__ void nvfp4_kernel_body(const Nvfp4Params& p) {
       acc_phase ^= 1u;
       const int row = u.row0 + r;
       const int col0 = u.n0 + half * 128;
-      if (row >= u.row_lo && row < u.row_hi && col0 < p.N) {
+      if (CG == 2 && u.row_lo <= u.row0 && u.row_hi >= u.row0 + BM && col0 < p.N) {
+        // every row of this CTA belongs to the unit's segment: two TMA stores of 32 rows x 64 columns
+        // per warp through a 128B-swizzled staging tile (columns past N are clipped by the store)
+        const uint32_t sbase = smem_u32(s.stage_c[warp]);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (col0 + 64 * c >= p.N) break;               // warp-uniform: the chunk lies past N
+          if (lane == 0) bulk_wait_read0();            // the previous store has read the tile
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(sbase + lane * 128 + ((j ^ (lane & 7)) << 4), o[32 * c + 4 * j], o[32 * c + 4 * j + 1],
+                         o[32 * c + 4 * j + 2], o[32 * c + 4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&p.tmC, s.stage_c[warp], (col0 + 64 * c) * 2, u.row0 + quarter * 32);
+            bulk_commit();
+          }
+        }
+      } else if (row >= u.row_lo && row < u.row_hi && col0 < p.N) {
         const int ncols = min(128, p.N - col0);
         __nv_bfloat16* dst = p.C + static_cast<size_t>(row) * p.N + col0;
 #pragma unroll
@@ -393,6 +435,7 @@ __device__ __forceinline__ void nvfp4_kernel_body(const Nvfp4Params& p) {
     }
   }
 
+  if (CG == 2 && warp < EPI_WARPS && lane == 0) bulk_wait0();   // this warp's TMA stores are complete
   tc_fence_before();
   if (CG == 2) {
     cluster_sync();  // the even CTA's MMAs into the odd CTA's TMEM are complete (mma_done waited)
