@@ -129,7 +129,7 @@ template <int CG>
 constexpr size_t smem_bytes() {
   return sizeof(Smem<CG>) + 1024;  // + alignment slack
 }
-static_assert(smem_bytes<2>() <= 232448, "pair kernel shared memory above 227 KB");
+static_assert(smem_bytes<1>() <= 232448 && smem_bytes<2>() <= 232448, "nvfp4 kernels' shared memory above 227 KB");
 
 template <int CG>
 __device__ __forceinline__ Smem<CG>& smem_ref(uint8_t* raw) {
