@@ -61,3 +61,30 @@ def test_bracketing_products_enclose_the_quotient():
             q_hi = rn32(F(x) * F(rn32(F(r) * F(hi_f))))
             lo, hi = (q_lo, q_hi) if x >= 0 else (q_hi, q_lo)
             assert lo <= q <= hi
+
+
+def test_bracket_codes_differ_by_at_most_one_without_borrow():
+    """The kernels take their flags from (packed codes of x r(1 + 2^-21)) - (packed codes of
+    x r(1 - 2^-21)): this needs every element's two codes to be equal or adjacent, the larger one from
+    the larger product, with the same sign bit -- checked here with the input generators' encoders on
+    products spread over every binade of both formats (near cell boundaries included)."""
+    from nvfp4_grouped_gemm_indices_b200 import workloads as W
+
+    rng = np.random.default_rng(11)
+    lo_f, hi_f = np.float32(1 - 2.0 ** -21), np.float32(1 + 2.0 ** -21)
+    # magnitudes across the whole code range, plus exact midpoints and their fp32 neighbours
+    mags = np.concatenate([
+        np.float32(2.0) ** rng.uniform(-12, 9.2, 20000).astype(np.float32),
+        np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 2.0 ** -10, 1.0625, 464.0, 0.0], np.float32),
+    ]).astype(np.float32)
+    mags = np.concatenate([mags, np.nextafter(mags, np.float32(0)), np.nextafter(mags, np.float32(1e9))])
+    q = (mags * rng.choice(np.array([-1, 1], np.float32), mags.size)).astype(np.float32)
+    q_lo = (q * lo_f).astype(np.float32)
+    q_hi = (q * hi_f).astype(np.float32)
+    for enc, sign_bit in ((W.e4m3_encode, 0x80), (W.e2m1_encode, 0x8)):
+        c_lo = enc(q_lo).astype(np.int32)
+        c_hi = enc(q_hi).astype(np.int32)
+        assert np.array_equal(c_lo & sign_bit, c_hi & sign_bit)           # same sign bit
+        d = c_hi - c_lo                                                   # magnitude codes: no borrow
+        assert d.min() >= 0 and d.max() <= 1
+        assert d.sum() > 0                                                # the boundary cases occur
