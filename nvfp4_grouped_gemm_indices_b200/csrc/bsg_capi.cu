@@ -205,6 +205,39 @@ bsg_status check_common(const void* A, const void* B, const int32_t* m_indices, 
   return BSG_OK;
 }
 
+
+// One GEMM launch through cudaLaunchKernelEx.  A grid smaller than the GPU (a small problem) is
+// launched as a programmatic dependent of the previous kernel on the stream: its CTAs start on the
+// idle SMs and do their set-up (barriers, TMEM, descriptor prefetch) while that kernel finishes, and
+// wait for it on the device before touching memory (the FP8 page's M=65 shape: 5.5 -> 4.5 us per
+// launch under graph replay).  Full-GPU grids keep plain stream order.  `pair`: 2-CTA clusters.
+template <typename Kern, typename Params>
+cudaError_t launch_gemm(Kern kernel, int grid, int threads, size_t smem, cudaStream_t cs, bool pair,
+                        int sm_count, const Params& p) {
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute la[2];
+  int n = 0;
+  if (grid < sm_count) {
+    la[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    la[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (pair) {
+    la[n].id = cudaLaunchAttributeClusterDimension;
+    la[n].val.clusterDim.x = 2;
+    la[n].val.clusterDim.y = 1;
+    la[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  lc.gridDim = dim3(grid, 1, 1);
+  lc.blockDim = dim3(threads, 1, 1);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = cs;
+  lc.attrs = la;
+  lc.numAttrs = n;
+  return cudaLaunchKernelEx(&lc, kernel, p);
+}
+
 // Raster groups of N tiles: when one expert's B (N x K bytes) fits comfortably in L2 the units run
 // window-major (all N tiles of a window together); otherwise N tiles are grouped so that the group's
 // slice of B (about 24 MB) stays resident while every window streams past it.
@@ -335,10 +368,12 @@ bsg_status fp8_swap_launch(DeviceState* dev, const void* A, const void* B, const
   const int grid = bsg_forced_grid(0, static_cast<int>(units < dev->sm_count ? units : dev->sm_count));
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if (nh == 1)
-    bsg::fp8s::bsg_fp8_swap_kernel<<<grid, bsg::fp8s::THREADS, bsg::fp8s::smem_bytes<1>(), cs>>>(p);
+    e = launch_gemm(bsg::fp8s::bsg_fp8_swap_kernel, grid, bsg::fp8s::THREADS, bsg::fp8s::smem_bytes<1>(), cs, false,
+                    dev->sm_count, p);
   else
-    bsg::fp8s::bsg_fp8_swap_n256_kernel<<<grid, bsg::fp8s::THREADS, bsg::fp8s::smem_bytes<2>(), cs>>>(p);
-  e = cudaGetLastError();
+    e = launch_gemm(bsg::fp8s::bsg_fp8_swap_n256_kernel, grid, bsg::fp8s::THREADS, bsg::fp8s::smem_bytes<2>(), cs,
+                    false, dev->sm_count, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launch of the fp8 swapped kernel");
   return BSG_OK;
 }
@@ -425,10 +460,12 @@ bsg_status fp8_launch(DeviceState* dev, const void* A, const void* B, const floa
       dev->fp8_n64_attr = true;
     }
     const int grid = bsg_forced_grid(0, grid_for(dev->sm_count, M, N, G, bn));
-    bsg::fp8::bsg_fp8_grouped_n64_kernel<<<grid, bsg::fp8::THREADS, bsg::fp8::smem_bytes<1, 64>(), cs>>>(p);
+    e = launch_gemm(bsg::fp8::bsg_fp8_grouped_n64_kernel, grid, bsg::fp8::THREADS, bsg::fp8::smem_bytes<1, 64>(), cs,
+                    false, dev->sm_count, p);
   } else if (cg == 1) {
     const int grid = bsg_forced_grid(0, grid_for(dev->sm_count, M, N, G, bn));
-    bsg::fp8::bsg_fp8_grouped_kernel<<<grid, bsg::fp8::THREADS, bsg::fp8::smem_bytes<1>(), cs>>>(p);
+    e = launch_gemm(bsg::fp8::bsg_fp8_grouped_kernel, grid, bsg::fp8::THREADS, bsg::fp8::smem_bytes<1>(), cs, false,
+                    dev->sm_count, p);
   } else {
     if (dev->fp8_pair_clusters < 1) return fail(BSG_ERR_CUDA, "no SM-pair cluster fits on this device");
     const BsgUnitEstimate est = bsg_estimate_units(M, G);
@@ -436,22 +473,11 @@ bsg_status fp8_launch(DeviceState* dev, const void* A, const void* B, const floa
     int64_t clusters = est.pairs_max * n_tiles;
     if (clusters > dev->fp8_pair_clusters) clusters = dev->fp8_pair_clusters;
     const int grid = 2 * ((bsg_forced_grid(0, static_cast<int>(2 * clusters)) + 1) / 2);
-    cudaLaunchConfig_t lc = {};
-    cudaLaunchAttribute la[1];
-    la[0].id = cudaLaunchAttributeClusterDimension;
-    la[0].val.clusterDim.x = 2;
-    la[0].val.clusterDim.y = 1;
-    la[0].val.clusterDim.z = 1;
-    lc.gridDim = dim3(grid, 1, 1);
-    lc.blockDim = dim3(bsg::fp8::THREADS, 1, 1);
-    lc.dynamicSmemBytes = bsg::fp8::smem_bytes<2>();
-    lc.stream = cs;
-    lc.attrs = la;
-    lc.numAttrs = 1;
-    e = cudaLaunchKernelEx(&lc, bsg::fp8::bsg_fp8_grouped_2sm_kernel, p);
+    e = launch_gemm(bsg::fp8::bsg_fp8_grouped_2sm_kernel, grid, bsg::fp8::THREADS, bsg::fp8::smem_bytes<2>(), cs, true,
+                    dev->sm_count, p);
     if (e != cudaSuccess) return cuda_fail(e, "launch of the fp8 2-SM grouped kernel");
   }
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launch of the fp8 grouped kernel");
   return BSG_OK;
 }
@@ -557,7 +583,8 @@ bsg_status nvfp4_launch(DeviceState* dev, const void* A, const void* B, const vo
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if (cg == 1) {
     const int grid = bsg_forced_grid(1, grid_for(dev->sm_count, M, N, G, bsg::nvfp4::BN));
-    bsg::nvfp4::bsg_nvfp4_grouped_kernel<<<grid, bsg::nvfp4::THREADS, bsg::nvfp4::smem_bytes<1>(), cs>>>(p);
+    e = launch_gemm(bsg::nvfp4::bsg_nvfp4_grouped_kernel, grid, bsg::nvfp4::THREADS, bsg::nvfp4::smem_bytes<1>(), cs,
+                    false, dev->sm_count, p);
   } else {
     if (dev->nvfp4_pair_clusters < 1) return fail(BSG_ERR_CUDA, "no SM-pair cluster fits on this device");
     const BsgUnitEstimate est = bsg_estimate_units(M, G);
@@ -565,22 +592,11 @@ bsg_status nvfp4_launch(DeviceState* dev, const void* A, const void* B, const vo
     int64_t clusters = est.pairs_max * n_tiles;
     if (clusters > dev->nvfp4_pair_clusters) clusters = dev->nvfp4_pair_clusters;
     const int grid = 2 * ((bsg_forced_grid(1, static_cast<int>(2 * clusters)) + 1) / 2);
-    cudaLaunchConfig_t lc = {};
-    cudaLaunchAttribute la[1];
-    la[0].id = cudaLaunchAttributeClusterDimension;
-    la[0].val.clusterDim.x = 2;
-    la[0].val.clusterDim.y = 1;
-    la[0].val.clusterDim.z = 1;
-    lc.gridDim = dim3(grid, 1, 1);
-    lc.blockDim = dim3(bsg::nvfp4::THREADS, 1, 1);
-    lc.dynamicSmemBytes = bsg::nvfp4::smem_bytes<2>();
-    lc.stream = cs;
-    lc.attrs = la;
-    lc.numAttrs = 1;
-    e = cudaLaunchKernelEx(&lc, bsg::nvfp4::bsg_nvfp4_grouped_2sm_kernel, p);
+    e = launch_gemm(bsg::nvfp4::bsg_nvfp4_grouped_2sm_kernel, grid, bsg::nvfp4::THREADS, bsg::nvfp4::smem_bytes<2>(),
+                    cs, true, dev->sm_count, p);
     if (e != cudaSuccess) return cuda_fail(e, "launch of the nvfp4 2-SM kernel");
   }
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launch of the nvfp4 kernel");
   return BSG_OK;
 }

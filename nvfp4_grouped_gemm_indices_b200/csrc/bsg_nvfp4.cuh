@@ -194,6 +194,11 @@ __device__ __forceinline__ void nvfp4_kernel_body(const Nvfp4Params& p) {
   }
   tc_fence_after();
   const uint32_t tmem_base = s.tmem_base;
+  // Small launches run as programmatic dependents of the previous kernel on the stream: the set-up
+  // above overlapped it; wait for it to complete (its writes visible) before touching global memory,
+  // then let the next kernel start its own set-up.  Without that launch attribute both are no-ops.
+  grid_dependency_wait();
+  grid_dependents_launch();
 
   if (warp == WARP_SCHED) {
     run_scheduler<Q, BN, CG == 2>(s.queue, p.m_indices, p.M, p.G, n_tiles, p.n_group, wctx, p.debug_mode);
