@@ -227,7 +227,7 @@ def visible_gpu_index(local_rank):
 
 # The device code each workload's counters depend on: its kernels' own headers, the shared PTX
 # wrappers and scheduler, and the tactic chooser that picks among them.  A change anywhere else (host
-# entry points, another kernel family) leaves the recorded counters valid.
+# entry points, another kernel family, comments) leaves the recorded counters valid.
 KERNEL_SOURCES = {
     "fp8": ["bsg_fp8.cuh", "bsg_fp8_swap.cuh", "bsg_sched.cuh", "bsg_ptx.cuh", "bsg_chooser.cpp"],
     "nvfp4": ["bsg_nvfp4.cuh", "bsg_sched.cuh", "bsg_ptx.cuh", "bsg_chooser.cpp"],
@@ -241,12 +241,14 @@ def kernel_family(workload_name):
 
 
 def kernel_source_hash(family):
+    """Hash of the code (comments and blank lines removed) of a kernel family's sources."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "nvfp4_grouped_gemm_indices_b200", "csrc")
     for f in sorted(KERNEL_SOURCES[family]):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode())
-            h.update(fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            code = [line.split("//", 1)[0].rstrip() for line in fh]
+        h.update(f.encode())
+        h.update("\n".join(line for line in code if line).encode())
     return h.hexdigest()[:16]
 
 

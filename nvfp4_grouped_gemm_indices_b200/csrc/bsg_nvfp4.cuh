@@ -14,7 +14,11 @@
 //           the MMAs and commits to both CTAs' barriers.
 //   warps 0..7   epilogue: after the last K stage of a unit, read the 128 x BN FP32 accumulator from
 //                TMEM (warp w: lanes 32*(w%4).., columns 128*(w/4)..), scale by alpha[g] and pack to
-//                BF16 while reading, release the accumulator, then store the segment's rows.
+//                BF16 while reading, release the accumulator, then store the segment's rows: in the
+//                pair kernel, when all 128 rows of the CTA belong to the segment, through a per-warp
+//                128B-swizzled staging tile and TMA stores (2 x 32 rows x 64 columns); otherwise, and
+//                in the one-SM kernel (no shared memory left beside its ring), with masked 16-byte
+//                register stores.
 //   warp 8       TMA producer for A and B (K stage = 256 elements = 128 packed bytes, 128B swizzle);
 //                it also loads the stage's row-major scale bytes (sfa: 128 rows x 16 B, sfb: BN rows
 //                x 16 B) with TMA into a raw per-stage buffer.
