@@ -5,6 +5,9 @@
  * tcgen05 / TMA / TMEM kernels.  Everything is asynchronous on the caller's CUDA stream; nothing is
  * allocated, synchronised or retained by a call.  All pointers are CUDA device pointers owned by the
  * caller unless stated otherwise.  All tensors are dense, row-major, with no padding between rows.
+ * Stream order is kept: a GEMM launch whose grid is smaller than the GPU is a programmatic dependent
+ * of the previous kernel on the stream (it may start its set-up early) and waits on the device for
+ * that kernel to complete before it reads or writes any operand.
  *
  * Error convention (after the argument checks of the FP8 page's host binding, "[flashinfer]
  * FlashInfer FP8 GEMM 최적화: 윈도우 세그먼트 KG1 프로그램으로 GPU 성능 극대화", section 1): every entry
