@@ -894,8 +894,7 @@ bsg_status moe_launch(DeviceState* dev, const int32_t* expert_ids, int64_t T, in
   cudaLaunchAttribute la[1];
   la[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   la[0].val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t lc;
-  memset(&lc, 0, sizeof(lc));
+  cudaLaunchConfig_t lc = {};
   lc.stream = cs;
   lc.attrs = la;
   lc.numAttrs = 1;
